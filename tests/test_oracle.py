@@ -1,0 +1,327 @@
+"""Pins for the CPU oracle, none of which re-types its formulas.
+
+Each test compares the oracle with something fixed independently of it: a
+textbook library routine (torch scaled_dot_product_attention on CPU in
+float64), pure-Python brute force, closed forms, or invariants that the
+CalibAtt paper page fixes (Figure 3(b): a block kept for every prompt is
+always computed).  The cases are chosen so that a plausible slip -- a swapped
+block index, a dropped scale, a missing padding rule, an off-by-one in the
+top-k count, a wrong tie-break, a wrong vote comparison -- fails one of them.
+"""
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+RNG = np.random.default_rng(1234)
+
+
+def sdpa64(q, k, v, scale):
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)) for x in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], scale=scale)[0].numpy()
+
+
+# ----------------------------------------------------------------- O1 attention
+
+def test_all_ones_mask_is_dense_sdpa():
+    B, H, N, Np, d, blk = 2, 3, 45, 48, 16, 8
+    q, k, v = (RNG.standard_normal((B, H, Np, d)) for _ in range(3))
+    mask = np.ones((H, Np // blk, Np // blk), np.uint8)
+    scale = 0.37
+    O, L = oracle.masked_attention(q, k, v, mask, N, blk, blk, scale)
+    for b in range(B):
+        for h in range(H):
+            ref = sdpa64(q[b, h, :N], k[b, h, :N], v[b, h, :N], scale)
+            np.testing.assert_allclose(O[b, h, :N], ref, atol=1e-12, rtol=0)
+            s = scale * q[b, h, :N] @ k[b, h, :N].T
+            lse_ref = np.array([math.log(math.fsum(math.exp(x) for x in row)) for row in s])
+            np.testing.assert_allclose(L[b, h, :N], lse_ref, atol=1e-12, rtol=0)
+    assert np.all(O[:, :, N:] == 0) and np.all(np.isneginf(L[:, :, N:]))
+
+
+def brute_attention(q, k, v, mask, N, bq, bk, scale):
+    """Pure-Python loops; independent of numpy's linear algebra."""
+    Np, d = len(q), len(q[0])
+    O = [[0.0] * d for _ in range(Np)]
+    L = [float("-inf")] * Np
+    for i in range(N):
+        js = [j for j in range(N) if mask[i // bq][j // bk]]
+        if not js:
+            continue
+        s = [scale * math.fsum(q[i][t] * k[j][t] for t in range(d)) for j in js]
+        m = max(s)
+        p = [math.exp(x - m) for x in s]
+        z = math.fsum(p)
+        for t in range(d):
+            O[i][t] = math.fsum(p[a] * v[j][t] for a, j in enumerate(js)) / z
+        L[i] = m + math.log(z)
+    return np.array(O), np.array(L)
+
+
+@pytest.mark.parametrize("N,Np,bq,bk", [(13, 16, 4, 4), (30, 32, 8, 4), (7, 8, 4, 8)])
+def test_brute_force_small(N, Np, bq, bk):
+    H, d = 2, 5
+    q, k, v = (RNG.standard_normal((1, H, Np, d)) for _ in range(3))
+    mask = (RNG.random((H, Np // bq, Np // bk)) < 0.5).astype(np.uint8)
+    mask[0, 0, :] = 0           # an empty query-block row
+    scale = 0.8
+    O, L = oracle.masked_attention(q, k, v, mask, N, bq, bk, scale)
+    for h in range(H):
+        Ob, Lb = brute_attention(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), mask[h].tolist(), N, bq, bk, scale)
+        np.testing.assert_allclose(O[0, h], Ob, atol=1e-12, rtol=0)
+        np.testing.assert_array_equal(np.isneginf(L[0, h]), np.isneginf(Lb))
+        fin = np.isfinite(Lb)
+        np.testing.assert_allclose(L[0, h][fin], Lb[fin], atol=1e-12, rtol=0)
+
+
+def test_zero_query_gives_mean_of_kept_values():
+    # q = 0: every kept key scores 0, so O is the plain mean of the kept, real
+    # values and LSE = log(#kept real keys).  An asymmetric mask catches a
+    # swapped (query block, key block) index; a ragged N catches padding.
+    H, N, Np, d, bq, bk = 1, 22, 24, 3, 8, 4
+    q = np.zeros((1, H, Np, d))
+    k = RNG.standard_normal((1, H, Np, d))
+    v = RNG.standard_normal((1, H, Np, d))
+    mask = np.zeros((H, 3, 6), np.uint8)
+    mask[0, 0, [1, 5]] = 1
+    mask[0, 1, [0]] = 1
+    mask[0, 2, [2, 3, 5]] = 1
+    O, L = oracle.masked_attention(q, k, v, mask, N, bq, bk, 1.0)
+    for i in range(N):
+        keys = [j for j in range(N) if mask[0, i // bq, j // bk]]
+        np.testing.assert_allclose(O[0, 0, i], v[0, 0, keys].mean(axis=0), atol=1e-14)
+        assert L[0, 0, i] == pytest.approx(math.log(len(keys)), abs=1e-14)
+
+
+def test_block_diagonal_equals_independent_blocks():
+    H, N, Np, d, blk = 2, 40, 40, 6, 8
+    q, k, v = (RNG.standard_normal((1, H, Np, d)) for _ in range(3))
+    mask = np.stack([np.eye(Np // blk, dtype=np.uint8)] * H)
+    O, _ = oracle.masked_attention(q, k, v, mask, N, blk, blk, 0.5)
+    for h in range(H):
+        for b0 in range(0, N, blk):
+            sl = slice(b0, b0 + blk)
+            np.testing.assert_allclose(O[0, h, sl], sdpa64(q[0, h, sl], k[0, h, sl], v[0, h, sl], 0.5), atol=1e-12)
+
+
+def test_constant_value_block_and_skipped_blocks_are_inert():
+    H, N, Np, d, blk = 1, 32, 32, 4, 8
+    q, k, v = (RNG.standard_normal((1, H, Np, d)) for _ in range(3))
+    mask = np.zeros((H, 4, 4), np.uint8)
+    mask[0, :, 2] = 1                       # one kept key block per row
+    v2 = v.copy()
+    v2[0, 0, 16:24] = np.array([1.5, -2.0, 0.25, 7.0])
+    O, _ = oracle.masked_attention(q, k, v2, mask, N, blk, blk, 1.0)
+    np.testing.assert_allclose(O[0, 0, :N], np.tile([1.5, -2.0, 0.25, 7.0], (N, 1)), atol=1e-13)
+    # perturbing skipped keys/values changes nothing; perturbing kept ones does
+    k3, v3 = k.copy(), v.copy()
+    k3[0, 0, :16] += 5.0
+    v3[0, 0, 24:] -= 3.0
+    Oa, La = oracle.masked_attention(q, k, v, mask, N, blk, blk, 1.0)
+    Ob, Lb = oracle.masked_attention(q, k3, v3, mask, N, blk, blk, 1.0)
+    np.testing.assert_array_equal(Oa, Ob)
+    np.testing.assert_array_equal(La, Lb)
+    k4 = k.copy()
+    k4[0, 0, 17] += 1.0
+    Oc, _ = oracle.masked_attention(q, k4, v, mask, N, blk, blk, 1.0)
+    assert np.abs(Oc - Oa).max() > 1e-6
+
+
+def test_softmax_rows_sum_to_one():
+    # the oracle's output with V = I (d = N) is the probability matrix itself
+    H, N, blk = 1, 16, 4
+    q = RNG.standard_normal((1, H, N, N))
+    k = RNG.standard_normal((1, H, N, N))
+    v = np.eye(N)[None, None]
+    mask = (RNG.random((H, 4, 4)) < 0.6).astype(np.uint8)
+    mask[0, np.arange(4), np.arange(4)] = 1
+    P, _ = oracle.masked_attention(q, k, v, mask, N, blk, blk, 0.3)
+    np.testing.assert_allclose(P[0, 0].sum(axis=1), 1.0, atol=1e-12)
+    for i in range(N):
+        for j in range(N):
+            if not mask[0, i // blk, j // blk]:
+                assert P[0, 0, i, j] == 0.0
+
+
+# ----------------------------------------------------------------- O2 energy
+
+def test_energy_rows_sum_to_one_and_uniform_closed_form():
+    H, N, Np, d, blk = 2, 37, 40, 4, 8
+    q = RNG.standard_normal((H, Np, d))
+    k = RNG.standard_normal((H, Np, d))
+    E = oracle.block_energy(q, k, N, blk, blk, 0.7)
+    nq_real = math.ceil(N / blk)
+    np.testing.assert_allclose(E[:, :nq_real].sum(axis=2), 1.0, atol=1e-12)
+    # q = 0: uniform attention, E[qb, kb] = (#real keys in kb) / N
+    E0 = oracle.block_energy(np.zeros_like(q), k, N, blk, blk, 0.7)
+    counts = np.array([min(blk, max(0, N - kb * blk)) for kb in range(Np // blk)]) / N
+    np.testing.assert_allclose(E0[:, :nq_real], np.broadcast_to(counts, E0[:, :nq_real].shape), atol=1e-14)
+
+
+def test_energy_one_hot_closed_form():
+    # q = k = c * I: s_ii = scale * c^2, s_ij = 0 (i != j), so
+    # p_ii = e^a / (e^a + N - 1) and p_ij = 1 / (e^a + N - 1), a = scale * c^2.
+    N, blk, c, scale = 12, 4, 2.0, 0.5
+    q = (c * np.eye(N))[None]
+    E = oracle.block_energy(q, q.copy(), N, blk, blk, scale)
+    ea = math.exp(scale * c * c)
+    z = ea + N - 1
+    for qb in range(3):
+        for kb in range(3):
+            want = (ea + (blk - 1)) / z if qb == kb else blk / z
+            assert E[0, qb, kb] == pytest.approx(want, abs=1e-14)
+
+
+def test_energy_brute_force():
+    N, blk, d = 10, 4, 3
+    q = RNG.standard_normal((1, 12, d))
+    k = RNG.standard_normal((1, 12, d))
+    E = oracle.block_energy(q, k, N, blk, blk, 0.9)
+    for qb in range(3):
+        rows = [i for i in range(qb * blk, min(qb * blk + blk, N))]
+        for kb in range(3):
+            tot = 0.0
+            for i in rows:
+                s = [0.9 * math.fsum(q[0, i, t] * k[0, j, t] for t in range(d)) for j in range(N)]
+                z = math.fsum(math.exp(x) for x in s)
+                tot += math.fsum(math.exp(s[j]) / z for j in range(kb * blk, min(kb * blk + blk, N)))
+            assert E[0, qb, kb] == pytest.approx(tot / len(rows), abs=1e-13)
+
+
+# ----------------------------------------------------------------- O3 select
+
+def test_topk_count_and_brute_force_order():
+    assert oracle.topk_count(0.25, 256) == 64
+    assert oracle.topk_count(0.2, 591) == 119
+    assert oracle.topk_count(1e-9, 10) == 1
+    assert oracle.topk_count(1.0, 10) == 10
+    E = RNG.random((5, 7, 13))
+    E[0, 0, 3] = E[0, 0, 9]                # a tie
+    keep = oracle.select_topk(E, 0.3)
+    k = math.ceil(0.3 * 13)
+    assert np.all(keep.sum(axis=-1) == k)
+    for idx in np.ndindex(5, 7):
+        row = E[idx].tolist()
+        want = sorted(range(13), key=lambda j: (-row[j], j))[:k]
+        assert sorted(np.nonzero(keep[idx])[0].tolist()) == sorted(want)
+
+
+def test_topk_ties_keep_smallest_indices():
+    keep = oracle.select_topk(np.full((1, 10), 0.1), 0.35)
+    assert keep[0].tolist() == [1, 1, 1, 1, 0, 0, 0, 0, 0, 0]
+
+
+def test_energy_select_is_minimal_prefix_exact():
+    # dyadic energies: every partial sum is exact, so Fractions decide the answer
+    for trial in range(50):
+        r = np.random.default_rng(trial)
+        nkb = int(r.integers(1, 20))
+        vals = r.integers(0, 64, nkb)
+        E = (vals / 64.0)[None]
+        eps = float(r.choice([0.0, 0.25, 0.5, 0.125, 0.9]))
+        keep = oracle.select_energy(E, eps)[0]
+        order = sorted(range(nkb), key=lambda j: (-vals[j], j))
+        target = (1 - Fraction(eps)) * Fraction(int(vals.sum()), 64)
+        run, want = Fraction(0), set()
+        for j in order:
+            want.add(j)
+            run += Fraction(int(vals[j]), 64)
+            if run >= target:
+                break
+        assert set(np.nonzero(keep)[0].tolist()) == want
+
+
+# ----------------------------------------------------------------- O4 vote
+
+def test_min_votes_for():
+    assert oracle.min_votes_for(0.5, 8) == 4
+    assert oracle.min_votes_for(0.3, 10) == 3
+    assert oracle.min_votes_for(1.0, 7) == 7
+    assert oracle.min_votes_for(0.0, 7) == 0
+    assert oracle.min_votes_for(0.51, 8) == 5
+
+
+def test_vote_invariants():
+    I, H, nqb, nkb = 6, 3, 5, 9
+    keeps = (RNG.random((I, H, nqb, nkb)) < 0.4).astype(np.uint8)
+    keeps[:, 0, 0, 4] = 1                       # kept by every input
+    keeps[:, 1, 2, :] = 0                       # never kept -> guard must fire
+    keeps[0, 1, 2, 7] = 1                       # ... and pick the most-voted block
+    E = RNG.random((I, H, nqb, nkb)).astype(np.float32)
+    for mv in range(1, I + 1):
+        mask, votes, esum = oracle.vote(keeps, mv, E)
+        assert np.array_equal(votes, keeps.sum(axis=0))
+        allkept = keeps.all(axis=0)
+        assert np.all(mask[allkept] == 1)            # Figure 3(b): frequency 1 => computed
+        assert np.all(mask.sum(axis=-1) >= 1)
+        rowsempty = ~(votes >= mv).any(axis=-1)
+        plain = (votes >= mv).astype(np.uint8)
+        assert np.array_equal(mask[~rowsempty], plain[~rowsempty])
+        assert np.all(mask[rowsempty].sum(axis=-1) == 1)
+        assert mask[1, 2, 7] == 1 and mask[1, 2].sum() == 1
+    union, _, _ = oracle.vote(keeps, 1, E)
+    inter, _, _ = oracle.vote(keeps, I, E)
+    nonempty_u = keeps.any(axis=0).any(axis=-1)
+    assert np.array_equal(union[nonempty_u], keeps.any(axis=0).astype(np.uint8)[nonempty_u])
+    nonempty_i = keeps.all(axis=0).any(axis=-1)
+    assert np.array_equal(inter[nonempty_i], keeps.all(axis=0).astype(np.uint8)[nonempty_i])
+
+
+def test_vote_guard_tie_break():
+    keeps = np.zeros((2, 1, 1, 5), np.uint8)
+    keeps[0, 0, 0, 1] = 1
+    keeps[1, 0, 0, 3] = 1
+    E = np.zeros((2, 1, 1, 5), np.float32)
+    E[:, 0, 0, 3] = 0.25
+    E[:, 0, 0, 1] = 0.25
+    mask, _, _ = oracle.vote(keeps, 2, E)     # votes tie (1, 1); energy ties; smaller index wins
+    assert mask[0, 0].tolist() == [0, 1, 0, 0, 0]
+    E[1, 0, 0, 3] = 0.5
+    mask, _, _ = oracle.vote(keeps, 2, E)     # larger energy sum wins
+    assert mask[0, 0].tolist() == [0, 0, 0, 1, 0]
+
+
+# ----------------------------------------------------------------- O5 compile
+
+def test_compile_round_trip_and_counts():
+    masks = (RNG.random((4, 11, 13)) < 0.3).astype(np.uint8)
+    masks[1, 3] = 0
+    for dedup in (True, False):
+        bl = oracle.compile_blocklist(masks, dedup=dedup)
+        assert np.array_equal(oracle.expand_blocklist(bl), masks)
+        assert bl["nnz"] == int(masks.sum())
+        rows = masks.reshape(-1, 13)
+        for r in range(rows.shape[0]):
+            cols = bl["csr_col"][bl["csr_row_ptr"][r]:bl["csr_row_ptr"][r + 1]]
+            assert cols.tolist() == np.nonzero(rows[r])[0].tolist()
+        assert bl["row_pat"][1 * 11 + 3] == 0 and bl["pat_ptr"][0] == bl["pat_ptr"][1] == 0
+    bl = oracle.compile_blocklist(masks, dedup=False)
+    assert bl["n_pat"] == 1 + int((masks.reshape(-1, 13).sum(axis=1) > 0).sum())
+
+
+def test_compile_banded_closed_form():
+    # |qb - kb| <= w on an n x n grid: rows are translates of w + 1 distinct
+    # offset lists {0..L-1}, L = w+1 .. 2w+1 (top and bottom edge rows of equal
+    # length coincide), so n_pat = w + 2 with the empty pattern.
+    n, w = 20, 3
+    m = np.zeros((1, n, n), np.uint8)
+    for i in range(n):
+        m[0, i, max(0, i - w):min(n, i + w + 1)] = 1
+    bl = oracle.compile_blocklist(m)
+    assert bl["n_pat"] == w + 2
+    for p in range(1, w + 2):   # first occurrence order: row p-1 has length w + p
+        lst = bl["pat_off"][bl["pat_ptr"][p]:bl["pat_ptr"][p + 1]]
+        assert lst.tolist() == list(range(w + p))
+    assert bl["row_pat"][n - 1] == 1 and bl["row_base"][n - 1] == n - 1 - w
+
+
+def test_compile_empty_and_full():
+    bl = oracle.compile_blocklist(np.zeros((2, 3, 4), np.uint8))
+    assert bl["n_pat"] == 1 and bl["nnz"] == 0 and bl["nnz_pat"] == 0
+    bl = oracle.compile_blocklist(np.ones((2, 3, 4), np.uint8))
+    assert bl["n_pat"] == 2 and bl["nnz_pat"] == 4 and np.all(bl["row_pat"] == 1) and np.all(bl["row_base"] == 0)
