@@ -1,0 +1,284 @@
+"""Calibrated block-sparse spatiotemporal attention (CalibAtt) for B200.
+
+Thin Python binding over libcalibatt.so (C ABI: ``include/calibatt.h``).
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks and marshals arguments, allocates outputs and workspace with
+PyTorch, and passes the current CUDA stream.  There is no CPU fallback: the
+functions raise if the library is missing or a tensor is not on a GPU.
+
+Method (arXiv 2603.05503, paper page): offline calibration scores key blocks
+per query block by their post-softmax energy (Figure 2, Table S5), keeps the
+top blocks (Figure 5(a)), votes them across calibration inputs with an
+agreement threshold (Figure 3(b), Figure 7), compiles the result into
+per-(layer, head, timestep) kept-block lists (Abstract), and at inference
+computes only the kept blocks (Abstract, Figure 5(b) top).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_ENERGY, SELECT_TOPK,
+                   CalibattError, check, load)
+
+__all__ = [
+    "BlockList", "sparse_attn_fwd", "block_energy", "select_vote", "finalize_mask", "calibrate",
+    "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
+    "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
+    "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
+]
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: use torch.bfloat16 or torch.float32")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def default_scale(d):
+    """float32 of 1/sqrt(d): the softmax scale the kernels multiply by."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+
+
+def launch_count():
+    """Kernel launches issued by the library so far in this process."""
+    return int(load().calibatt_launch_count())
+
+
+def min_votes_for(rho, n_inputs):
+    """Integer agreement threshold: keep a block iff votes / I >= rho."""
+    v = math.ceil(round(float(rho) * int(n_inputs), 9))
+    return int(min(max(v, 0), int(n_inputs)))
+
+
+def topk_count(frac, nkb):
+    """Kept key blocks per row in top-k mode: ceil(frac * nkb) clamped to [1, nkb]."""
+    return int(min(nkb, max(1, math.ceil(frac * nkb))))
+
+
+@dataclass
+class BlockList:
+    """Compiled kept-block lists on the GPU (see ``calibatt_blocklist``)."""
+
+    n_maps: int
+    n_q_blocks: int
+    n_k_blocks: int
+    block_q: int
+    block_k: int
+    row_base: torch.Tensor
+    row_pat: torch.Tensor
+    pat_ptr: torch.Tensor
+    pat_off: torch.Tensor
+    csr_row_ptr: torch.Tensor | None
+    csr_col: torch.Tensor | None
+    n_pat: int
+    nnz_pat: int
+    nnz: int
+
+    def as_struct(self):
+        s = _lib.Blocklist()
+        s.n_maps, s.n_q_blocks, s.n_k_blocks = self.n_maps, self.n_q_blocks, self.n_k_blocks
+        s.block_q, s.block_k = self.block_q, self.block_k
+        s.row_base = self.row_base.data_ptr()
+        s.row_pat = self.row_pat.data_ptr()
+        s.pat_ptr = self.pat_ptr.data_ptr()
+        s.pat_off = self.pat_off.data_ptr() if self.pat_off.numel() else None
+        s.csr_row_ptr = self.csr_row_ptr.data_ptr() if self.csr_row_ptr is not None else None
+        s.csr_col = self.csr_col.data_ptr() if self.csr_col is not None and self.csr_col.numel() else None
+        s.n_pat, s.nnz_pat, s.nnz = self.n_pat, self.nnz_pat, self.nnz
+        return s
+
+    def to_numpy(self):
+        out = {k: getattr(self, k) for k in ("n_maps", "n_q_blocks", "n_k_blocks", "n_pat", "nnz_pat", "nnz")}
+        for k in ("row_base", "row_pat", "pat_ptr", "pat_off", "csr_row_ptr", "csr_col"):
+            v = getattr(self, k)
+            out[k] = v.cpu().numpy() if v is not None else None
+        return out
+
+    @property
+    def density(self):
+        return self.nnz / float(self.n_maps * self.n_q_blocks * self.n_k_blocks)
+
+    def kept_blocks(self, map_offset=0, n=None):
+        """Kept blocks of maps [map_offset, map_offset + n): computed on the GPU from the pattern pool."""
+        n = self.n_maps - map_offset if n is None else n
+        r0, r1 = map_offset * self.n_q_blocks, (map_offset + n) * self.n_q_blocks
+        lens = self.pat_ptr[1:] - self.pat_ptr[:-1]
+        return int(lens[self.row_pat[r0:r1].long()].sum().item())
+
+
+def sparse_attn_fwd(q, k, v, bl: BlockList, N, scale=None, map_offset=0, return_lse=False, out=None, lse=None,
+                    status=None):
+    """Block-sparse attention forward.  q, k, v: [B, H, Np, d] bf16 or fp32 on the GPU.
+
+    Returns O (and LSE [B, H, Np] fp32 when ``return_lse``).  ``status`` is an
+    optional int32 CUDA tensor that receives device-side error codes.
+    """
+    _need_cuda(q, k, v)
+    B, H, Np, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Np), device=q.device, dtype=torch.float32)
+    _need_cuda(out, lse, status)
+    s = bl.as_struct()
+    with torch.cuda.device(q.device):
+        check(load().calibatt_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, int(N), Np, d,
+                                              _dtype_code(q), scale, ctypes.byref(s), int(map_offset),
+                                              _ptr(status), _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def _calib_workspace(H, N, Np, d, bq, bk, device):
+    n = ctypes.c_size_t(0)
+    check(load().calibatt_calibrate_workspace_size(H, int(N), Np, d, bq, bk, ctypes.byref(n)))
+    return torch.empty(n.value, dtype=torch.uint8, device=device)
+
+
+def block_energy(q, k, N, block_q=128, block_k=128, scale=None, status=None, workspace=None):
+    """Block energies [H, nqb, nkb] fp32 of one input; q, k: [H, Np, d]."""
+    _need_cuda(q, k)
+    H, Np, d = q.shape
+    scale = default_scale(d) if scale is None else float(scale)
+    E = torch.empty((H, Np // block_q, Np // block_k), device=q.device, dtype=torch.float32)
+    ws = _calib_workspace(H, N, Np, d, block_q, block_k, q.device) if workspace is None else workspace
+    with torch.cuda.device(q.device):
+        check(load().calibatt_block_energy(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q, block_k,
+                                           scale, _ptr(E), _ptr(ws), ws.numel(), _ptr(status), _stream(q.device)))
+    return E
+
+
+def select_vote(energy, mode, param, votes, energy_sum):
+    """Adds one input's selection (top-k fraction or energy eps) into votes / energy_sum (in place)."""
+    _need_cuda(energy, votes, energy_sum)
+    H, nqb, nkb = energy.shape
+    with torch.cuda.device(energy.device):
+        check(load().calibatt_select_vote(_ptr(energy), H, nqb, nkb, int(mode), float(param), _ptr(votes),
+                                          _ptr(energy_sum), _stream(energy.device)))
+    return votes, energy_sum
+
+
+def finalize_mask(votes, energy_sum, min_votes):
+    """uint8 mask [H, nqb, nkb] = votes >= min_votes, with the empty-row guard."""
+    _need_cuda(votes, energy_sum)
+    H, nqb, nkb = votes.shape
+    mask = torch.empty((H, nqb, nkb), dtype=torch.uint8, device=votes.device)
+    with torch.cuda.device(votes.device):
+        check(load().calibatt_finalize_mask(_ptr(votes), _ptr(energy_sum), H, nqb, nkb, int(min_votes), _ptr(mask),
+                                            _stream(votes.device)))
+    return mask
+
+
+def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mode=SELECT_TOPK, select_param=0.25,
+              rho=0.5, min_votes=None, votes=None, energy_sum=None, finalize=True, status=None):
+    """Calibration pass.  Returns (mask or None, votes, energy_sum).
+
+    ``votes`` / ``energy_sum`` (int32 / fp32 [H, nqb, nkb]) accumulate across
+    calls, so calibration can resume; ``min_votes`` defaults to
+    ceil(rho * total inputs seen), the total taken from ``votes``' callers.
+    """
+    n = len(q_list)
+    if n != len(k_list) or n == 0:
+        raise ValueError("need the same non-zero number of q and k tensors")
+    _need_cuda(*q_list, *k_list)
+    H, Np, d = q_list[0].shape
+    dev = q_list[0].device
+    nqb, nkb = Np // block_q, Np // block_k
+    scale = default_scale(d) if scale is None else float(scale)
+    if votes is None:
+        votes = torch.zeros((H, nqb, nkb), dtype=torch.int32, device=dev)
+    if energy_sum is None:
+        energy_sum = torch.zeros((H, nqb, nkb), dtype=torch.float32, device=dev)
+    if min_votes is None:
+        min_votes = min_votes_for(rho, n)
+    mask = torch.empty((H, nqb, nkb), dtype=torch.uint8, device=dev) if finalize else None
+    ws = _calib_workspace(H, N, Np, d, block_q, block_k, dev)
+    qp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in q_list])
+    kp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in k_list])
+    with torch.cuda.device(dev):
+        check(load().calibatt_calibrate(qp, kp, n, H, int(N), Np, d, _dtype_code(q_list[0]), block_q, block_k, scale,
+                                        int(select_mode), float(select_param), _ptr(votes), _ptr(energy_sum),
+                                        int(min_votes), _ptr(mask), _ptr(ws), ws.numel(), _ptr(status),
+                                        _stream(dev)))
+    return mask, votes, energy_sum
+
+
+def _compile_ws(n_maps, nqb, nkb, dev):
+    n = ctypes.c_size_t(0)
+    check(load().calibatt_compile_workspace_size(n_maps, nqb, nkb, ctypes.byref(n)))
+    return torch.empty(n.value, dtype=torch.uint8, device=dev)
+
+
+def compile_size(masks, dedup=DEDUP_HASH, workspace=None):
+    """(nnz, n_pat, nnz_pat) of compiling ``masks`` [n_maps, nqb, nkb] uint8 (synchronizes)."""
+    _need_cuda(masks)
+    n_maps, nqb, nkb = masks.shape
+    ws = _compile_ws(n_maps, nqb, nkb, masks.device) if workspace is None else workspace
+    nnz, n_pat, nnz_pat = ctypes.c_int64(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    with torch.cuda.device(masks.device):
+        check(load().calibatt_compile_size(_ptr(masks), n_maps, nqb, nkb, int(dedup), ctypes.byref(nnz),
+                                           ctypes.byref(n_pat), ctypes.byref(nnz_pat), _ptr(ws), ws.numel(),
+                                           _stream(masks.device)))
+    return nnz.value, n_pat.value, nnz_pat.value
+
+
+def compile(masks, block_q=128, block_k=128, dedup=DEDUP_HASH, with_csr=True):
+    """Compiles uint8 masks [n_maps, nqb, nkb] into a :class:`BlockList` (synchronizes)."""
+    _need_cuda(masks)
+    if masks.dtype != torch.uint8:
+        raise TypeError("masks must be uint8")
+    n_maps, nqb, nkb = masks.shape
+    dev = masks.device
+    ws = _compile_ws(n_maps, nqb, nkb, dev)
+    nnz, n_pat, nnz_pat = compile_size(masks, dedup, ws)
+    R = n_maps * nqb
+    bl = BlockList(
+        n_maps, nqb, nkb, block_q, block_k,
+        row_base=torch.empty(R, dtype=torch.int32, device=dev),
+        row_pat=torch.empty(R, dtype=torch.int32, device=dev),
+        pat_ptr=torch.empty(n_pat + 1, dtype=torch.int32, device=dev),
+        pat_off=torch.empty(max(nnz_pat, 1), dtype=torch.int16, device=dev)[:nnz_pat],
+        csr_row_ptr=torch.empty(R + 1, dtype=torch.int64, device=dev) if with_csr else None,
+        csr_col=torch.empty(max(nnz, 1), dtype=torch.int16, device=dev)[:nnz] if with_csr else None,
+        n_pat=n_pat, nnz_pat=nnz_pat, nnz=nnz,
+    )
+    s = bl.as_struct()
+    if nnz_pat == 0:
+        s.pat_off = None
+    with torch.cuda.device(dev):
+        check(load().calibatt_compile(_ptr(masks), n_maps, nqb, nkb, int(dedup), block_q, block_k, ctypes.byref(s),
+                                      _ptr(ws), ws.numel(), _stream(dev)))
+    return bl
+
+
+def selftest_wait_timeout(limit_ns=10_000_000, device=None):
+    """Runs the never-completing bounded wait; returns the device status (CALIBATT_E_TIMEOUT expected)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        check(load().calibatt_selftest_wait_timeout(int(limit_ns), _ptr(status), _stream(dev)))
+    return int(status.item())

@@ -1,0 +1,244 @@
+/*
+ * calibatt.h -- C ABI of the calibrated block-sparse attention library.
+ *
+ * The method is CalibAtt, "Accelerating Text-to-Video Generation with
+ * Calibrated Sparse Attention" (arXiv 2603.05503, paper page): an offline
+ * calibration pass finds block-level sparsity that is stable across inputs
+ * (Abstract; Figure 5(a)), the patterns are compiled into per-(layer, head,
+ * timestep) attention operations (Abstract), and at inference only the kept
+ * blocks are computed while the others are skipped (Abstract; Figure 5(b)
+ * top).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is caller-owned DEVICE memory unless marked
+ *    "host".  The library allocates no device memory: scratch comes from the
+ *    caller through (workspace, workspace_bytes), sized by the matching
+ *    *_workspace_size query.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  The only calls that synchronize the stream
+ *    are calibatt_compile_size and calibatt_compile (they read counts back).
+ *  - Every call returns a status: CALIBATT_OK (0) or a negative code below.
+ *    On a non-zero return nothing was launched unless the code is
+ *    CALIBATT_E_CUDA (a launch error).  calibatt_last_error() returns a
+ *    thread-local, human-readable description of the last failure.
+ *  - Errors found on the device (a corrupt block list, a bounded wait that
+ *    ran out) are written, first error wins, to the optional int32 device
+ *    word `dev_status` (0 = no error); the kernel then skips the affected
+ *    work and exits cleanly.  Nothing in the library asserts, traps or
+ *    aborts.
+ *  - Tensor layouts are row-major and contiguous.  Attention tensors are
+ *    [B, H, Np, d] with Np the padded sequence length (a multiple of the
+ *    block size) and N <= Np the real length; padding rows must be present
+ *    in memory (their values are ignored for keys and overwritten for
+ *    outputs).
+ */
+#ifndef CALIBATT_H
+#define CALIBATT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (binary-compatible with cudaStream_t / CUstream). */
+typedef struct CUstream_st* calibatt_stream_t;
+
+/* ---- status codes ---------------------------------------------------- */
+#define CALIBATT_OK              0
+#define CALIBATT_E_INVALID      -1 /* bad argument (null, size, alignment, range) */
+#define CALIBATT_E_UNSUPPORTED  -2 /* valid but not implemented (dtype/d/block)   */
+#define CALIBATT_E_CUDA         -3 /* a CUDA runtime/driver call failed           */
+#define CALIBATT_E_TIMEOUT      -4 /* a bounded device-side wait ran out          */
+#define CALIBATT_E_CORRUPT      -5 /* block list failed its device-side checks    */
+#define CALIBATT_E_WORKSPACE    -6 /* workspace missing or too small              */
+
+/* ---- element types and selection modes ------------------------------- */
+#define CALIBATT_BF16 0 /* bfloat16 inputs/outputs, tensor-core path           */
+#define CALIBATT_FP32 1 /* float32 inputs/outputs, CUDA-core (FFMA) path       */
+
+#define CALIBATT_SELECT_TOPK   0 /* keep ceil(frac * nkb) blocks (param = frac)  */
+#define CALIBATT_SELECT_ENERGY 1 /* keep energy mass >= 1 - eps (param = eps)    */
+
+#define CALIBATT_DEDUP_NONE 0 /* every non-empty row gets its own pattern       */
+#define CALIBATT_DEDUP_HASH 1 /* translation-relative row-pattern dedup         */
+#define CALIBATT_DEDUP_HASH_WEAK 2 /* same result, deliberately weak hash that
+                                      collides often (exercises the exact
+                                      collision path; for testing)             */
+
+/*
+ * Compiled kept-block lists (the mask dictionary in compiled form).
+ *
+ * Rows are (map, query block) pairs in map-major order, row r = map * nqb +
+ * qb, where a map is one (layer, timestep, head) mask with map id
+ * (layer * T + timestep) * H + head.  Row r keeps the key blocks
+ *     row_base[r] + pat_off[pat_ptr[p] .. pat_ptr[p+1]),  p = row_pat[r],
+ * ascending.  Pattern 0 is the empty pattern (a row with no kept block has
+ * row_base 0 and row_pat 0).  Offsets within a pattern are ascending and
+ * the first is 0.  Rows that are translates of one another share a pattern
+ * (the within-frame row repetition of the paper page's Figure 4(b)).
+ * The plain CSR (csr_row_ptr, csr_col) is optional (NULL to skip).
+ *
+ * All pointer members are device pointers owned by the caller.  Integer
+ * members are host values.
+ */
+typedef struct calibatt_blocklist {
+  int32_t n_maps, n_q_blocks, n_k_blocks, block_q, block_k;
+  int32_t* row_base;    /* [n_maps * n_q_blocks]                          */
+  int32_t* row_pat;     /* [n_maps * n_q_blocks]                          */
+  int32_t* pat_ptr;     /* [n_pat + 1]                                    */
+  int16_t* pat_off;     /* [nnz_pat]                                      */
+  int64_t* csr_row_ptr; /* [n_maps * n_q_blocks + 1] or NULL              */
+  int16_t* csr_col;     /* [nnz] or NULL                                  */
+  int32_t n_pat, nnz_pat;
+  int64_t nnz;
+} calibatt_blocklist;
+
+/* Thread-local text of the last error (never NULL). */
+const char* calibatt_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int calibatt_version(void);
+
+/* Number of kernel launches the library has issued in this process. */
+uint64_t calibatt_launch_count(void);
+
+/* Limit (nanoseconds) of every bounded device-side wait; default 2e9.
+ * Also read once from the environment variable CALIBATT_SPIN_LIMIT_NS.     */
+void calibatt_set_spin_limit_ns(uint64_t ns);
+uint64_t calibatt_get_spin_limit_ns(void);
+
+/*
+ * calibatt_sparse_attn_fwd -- block-sparse attention forward.
+ *
+ * Paper page, Abstract ("compute the selected input-dependent connections
+ * densely, and skip the unselected ones") and Figure 5(b) top (load the block
+ * mask, skip the unset blocks).  For batch b, head h and real query row
+ * i < N of query block qb = i / block_q, with map = map_offset + h:
+ *     J(i)  = { j < N : block j / block_k is kept in row (map, qb) of bl }
+ *     O_i   = sum_{j in J(i)} exp(scale q_i.k_j - m_i) v_j / sum_{j in J(i)} exp(scale q_i.k_j - m_i)
+ *     LSE_i = m_i + ln sum_{j in J(i)} exp(scale q_i.k_j - m_i),   m_i = max_j scale q_i.k_j
+ * Rows i >= N and rows whose J(i) is empty get O_i = 0, LSE_i = -inf.
+ *
+ *  q, k, v  [B, H, Np, d] of `dtype` (16-byte aligned); o the same shape
+ *           and type (written); lse [B, H, Np] float32 or NULL.
+ *  scale    the softmax scale (normally the float32 of 1/sqrt(d)).
+ *  bl       host pointer to a compiled block list with block_q = block_k
+ *           and n_q_blocks = n_k_blocks = Np / block_q;
+ *           map_offset + H <= bl->n_maps.  The mask is shared by the batch.
+ *  dev_status optional device int32 (see conventions).
+ * Supported: CALIBATT_BF16 with d in {64, 128}, block 128 (tcgen05 tensor
+ * cores, fp32 accumulation, P rounded to bf16 for the PV product);
+ * CALIBATT_FP32 with d in {64, 128}, block in {64, 128} (FFMA).  Anything
+ * else returns CALIBATT_E_UNSUPPORTED.
+ */
+int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int N, int Np, int d, int dtype, float scale,
+                             const calibatt_blocklist* bl, int map_offset,
+                             int32_t* dev_status, calibatt_stream_t stream);
+
+/*
+ * calibatt_block_energy -- block energies of one calibration input.
+ *
+ * Paper page, Figure 2 (block-level post-softmax attention maps) and
+ * Table S5 ("block energies"):
+ *     E[h, qb, kb] = (1 / #rows(qb)) sum_{i in qb, i < N} sum_{j in kb, j < N} softmax_j(scale q_i.k_j)
+ * with the softmax over ALL keys j < N (dense, unmasked).  Every row of E
+ * sums to 1.
+ *  q, k       [H, Np, d] of `dtype`;  energy_out [H, Np/block_q, Np/block_k] float32.
+ *  workspace  >= calibatt_calibrate_workspace_size bytes (256-byte aligned).
+ * Supported: CALIBATT_BF16 with d in {64,128}, blocks 128 (tensor cores);
+ * CALIBATT_FP32 with d in {64,128}, blocks in {64,128} (FFMA).
+ */
+int calibatt_block_energy(const void* q, const void* k, int H, int N, int Np, int d, int dtype,
+                          int block_q, int block_k, float scale, float* energy_out,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                          calibatt_stream_t stream);
+
+/* Workspace bytes needed by calibatt_block_energy / calibatt_calibrate. */
+int calibatt_calibrate_workspace_size(int H, int N, int Np, int d, int block_q, int block_k,
+                                      size_t* bytes);
+
+/*
+ * calibatt_select_vote -- per-row selection of one input's energies, added
+ * into the vote counts.
+ *
+ * Paper page, Figure 5(a) (threshold the top key blocks per query block) and
+ * Figure 3(b) (how often each block is kept across calibration prompts).
+ * Per row (h, qb), key blocks are ordered by (energy descending, index
+ * ascending).  TOPK keeps the first k = min(nkb, max(1, ceil(frac * nkb)));
+ * ENERGY keeps the shortest prefix whose float64 running sum reaches
+ * (1 - eps) * (float64 sum of the row in index order), the crossing block
+ * included.  Then votes[h,qb,kb] += kept and energy_sum[h,qb,kb] += E
+ * (float32).
+ *  energy      [H, nqb, nkb] float32 (read);  votes_inout int32, energy_sum_inout
+ *              float32, both [H, nqb, nkb] (read-modify-write).
+ */
+int calibatt_select_vote(const float* energy, int H, int nqb, int nkb, int select_mode,
+                         double select_param, int32_t* votes_inout, float* energy_sum_inout,
+                         calibatt_stream_t stream);
+
+/*
+ * calibatt_finalize_mask -- agreement threshold (paper page, Figure 7, rho).
+ * mask = votes >= min_votes.  A row left empty keeps exactly one key block:
+ * the one with the most votes, then the largest energy_sum, then the
+ * smallest index.  mask_out [H, nqb, nkb] uint8 (0/1).
+ */
+int calibatt_finalize_mask(const int32_t* votes, const float* energy_sum, int H, int nqb, int nkb,
+                           int min_votes, uint8_t* mask_out, calibatt_stream_t stream);
+
+/*
+ * calibatt_calibrate -- the calibration pass over n_inputs inputs.
+ *
+ * For each input: calibatt_block_energy, then calibatt_select_vote into
+ * votes_inout / energy_sum_inout (so repeated calls resume calibration:
+ * the counts simply add up).  If mask_out != NULL, finishes with
+ * calibatt_finalize_mask(min_votes).
+ *  q_list, k_list  HOST arrays of n_inputs device pointers, each [H, Np, d].
+ */
+int calibatt_calibrate(const void* const* q_list, const void* const* k_list, int n_inputs,
+                       int H, int N, int Np, int d, int dtype, int block_q, int block_k,
+                       float scale, int select_mode, double select_param,
+                       int32_t* votes_inout, float* energy_sum_inout, int min_votes,
+                       uint8_t* mask_out, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, calibatt_stream_t stream);
+
+/*
+ * Compile masks [n_maps, nqb, nkb] (uint8, non-zero = kept) into a
+ * calibatt_blocklist (paper page, Abstract: the patterns are compiled into
+ * attention operations for each layer, head and timestep).  Patterns are
+ * numbered in order of first occurrence over rows scanned in ascending
+ * order; pattern 0 is the empty pattern.  nkb must be <= 32767.
+ *
+ * Two phases.  calibatt_compile_size computes the sizes (nnz = kept blocks,
+ * n_pat = patterns incl. the empty one, nnz_pat = pattern-pool length) and
+ * synchronizes the stream.  The caller then allocates the arrays, sets the
+ * pointer members and the capacities n_pat / nnz_pat / nnz of `out`, and
+ * calls calibatt_compile, which fills them, writes n_maps .. block_k, and
+ * synchronizes; it fails with CALIBATT_E_INVALID if the capacities are
+ * smaller than the sizes.  Workspace: calibatt_compile_workspace_size.
+ */
+int calibatt_compile_workspace_size(int n_maps, int nqb, int nkb, size_t* bytes);
+int calibatt_compile_size(const uint8_t* masks, int n_maps, int nqb, int nkb, int dedup,
+                          int64_t* nnz, int32_t* n_pat, int32_t* nnz_pat,
+                          void* workspace, size_t workspace_bytes, calibatt_stream_t stream);
+int calibatt_compile(const uint8_t* masks, int n_maps, int nqb, int nkb, int dedup,
+                     int block_q, int block_k, calibatt_blocklist* out,
+                     void* workspace, size_t workspace_bytes, calibatt_stream_t stream);
+
+/*
+ * calibatt_selftest_wait_timeout -- launches one block that waits, with the
+ * bounded wait every kernel here uses, on a barrier that nothing completes.
+ * After `limit_ns` it gives up and writes CALIBATT_E_TIMEOUT to dev_status.
+ * Lets a caller check the timeout path without faulting or hanging a GPU.
+ */
+int calibatt_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status,
+                                   calibatt_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CALIBATT_H */

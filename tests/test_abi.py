@@ -1,0 +1,133 @@
+"""The C-ABI library loads, exports every function include/calibatt.h declares,
+and rejects bad arguments with status codes before touching the GPU.
+
+These run without a GPU: every call below fails validation on the host, so
+no CUDA call is made.
+"""
+
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from block_sparse_attention_cross_b200 import _lib
+
+HEADER = Path(__file__).resolve().parent.parent / "include" / "calibatt.h"
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = set(re.findall(r"\b(calibatt_[a-z_0-9]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_and_binding_agree():
+    names = declared_functions()
+    assert len(names) >= 14
+    assert set(names) == set(_lib.EXPORTS), set(names) ^ set(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_counters(lib):
+    assert lib.calibatt_version() == 10000
+    assert lib.calibatt_launch_count() == 0 or lib.calibatt_launch_count() > 0
+    old = lib.calibatt_get_spin_limit_ns()
+    assert old > 0
+    lib.calibatt_set_spin_limit_ns(12345)
+    assert lib.calibatt_get_spin_limit_ns() == 12345
+    lib.calibatt_set_spin_limit_ns(old)
+
+
+def _err(lib):
+    return lib.calibatt_last_error().decode()
+
+
+def test_fwd_rejects_null_and_bad_sizes(lib):
+    bl = _lib.Blocklist()
+    rc = lib.calibatt_sparse_attn_fwd(None, None, None, None, None, 1, 1, 128, 128, 128, _lib.BF16, 0.1,
+                                      ctypes.byref(bl), 0, None, None)
+    assert rc == _lib.E_INVALID and "non-NULL" in _err(lib)
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.calibatt_sparse_attn_fwd(fake, fake, fake, fake, None, 1, 1, 200, 128, 128, _lib.BF16, 0.1,
+                                      ctypes.byref(bl), 0, None, None)
+    assert rc == _lib.E_INVALID                       # Np < N
+    rc = lib.calibatt_sparse_attn_fwd(fake, fake, fake, fake, None, 1, 1, 128, 128, 128, _lib.BF16, -1.0,
+                                      ctypes.byref(bl), 0, None, None)
+    assert rc == _lib.E_INVALID and "scale" in _err(lib)
+    rc = lib.calibatt_sparse_attn_fwd(ctypes.c_void_p(0x10001), fake, fake, fake, None, 1, 1, 128, 128, 128,
+                                      _lib.BF16, 0.1, ctypes.byref(bl), 0, None, None)
+    assert rc == _lib.E_INVALID and "aligned" in _err(lib)
+    rc = lib.calibatt_sparse_attn_fwd(fake, fake, fake, fake, None, 1, 1, 128, 128, 128, _lib.BF16, 0.1,
+                                      None, 0, None, None)
+    assert rc == _lib.E_INVALID and "block list" in _err(lib)
+
+
+def _blocklist(n_maps, nq, nk, bq, bk):
+    bl = _lib.Blocklist()
+    bl.n_maps, bl.n_q_blocks, bl.n_k_blocks, bl.block_q, bl.block_k = n_maps, nq, nk, bq, bk
+    bl.row_base = bl.row_pat = bl.pat_ptr = bl.pat_off = 0x20000
+    bl.n_pat, bl.nnz_pat, bl.nnz = 1, 0, 0
+    return bl
+
+
+def test_fwd_rejects_mismatched_blocklist_and_unsupported(lib):
+    fake = ctypes.c_void_p(0x10000)
+    bl = _blocklist(2, 8, 8, 128, 128)
+    args = lambda B, H, N, Np, d, dt, mo: (fake, fake, fake, fake, None, B, H, N, Np, d, dt, 0.1,
+                                           ctypes.byref(bl), mo, None, None)
+    assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 1000, 1024, 128, _lib.BF16, 1)) == _lib.E_INVALID  # map range
+    assert "map_offset" in _err(lib)
+    assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 1000, 896, 128, _lib.BF16, 0)) == _lib.E_INVALID   # grid
+    assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 1000, 1024, 96, _lib.BF16, 0)) == _lib.E_UNSUPPORTED
+    assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 1000, 1024, 128, 7, 0)) == _lib.E_UNSUPPORTED
+    bl64 = _blocklist(2, 16, 16, 64, 64)
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, fake, None, 1, 2, 1024, 1024, 128, _lib.BF16, 0.1,
+                                        ctypes.byref(bl64), 0, None, None) == _lib.E_UNSUPPORTED
+    assert lib.calibatt_sparse_attn_fwd(fake, fake, fake, fake, None, 1, 2, 1024, 1024, 32, _lib.FP32, 0.1,
+                                        ctypes.byref(bl64), 0, None, None) == _lib.E_UNSUPPORTED
+    # padding of a whole block is rejected
+    assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 896, 1024, 128, _lib.BF16, 0)) == _lib.E_INVALID
+
+
+def test_workspace_queries(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.calibatt_calibrate_workspace_size(40, 32760, 32768, 128, 128, 128, ctypes.byref(n)) == _lib.OK
+    assert n.value >= 40 * 32768 * 4 + 40 * 256 * 256 * 4
+    assert lib.calibatt_calibrate_workspace_size(40, 32760, 32760, 128, 128, 128, ctypes.byref(n)) == _lib.E_INVALID
+    assert lib.calibatt_compile_workspace_size(4800, 256, 256, ctypes.byref(n)) == _lib.OK
+    assert n.value > 4800 * 256 * 8
+    assert lib.calibatt_compile_workspace_size(0, 256, 256, ctypes.byref(n)) == _lib.E_INVALID
+
+
+def test_calibration_and_compile_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.calibatt_block_energy(fake, fake, 2, 1000, 1024, 128, _lib.BF16, 64, 64, 0.1, fake, fake, 1 << 30,
+                                     None, None) == _lib.E_UNSUPPORTED
+    assert lib.calibatt_block_energy(fake, fake, 2, 1000, 1024, 128, _lib.BF16, 128, 128, 0.1, fake, fake, 16,
+                                     None, None) == _lib.E_WORKSPACE
+    assert lib.calibatt_select_vote(fake, 2, 8, 8, 5, 0.1, fake, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_TOPK, 0.0, fake, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_ENERGY, 1.0, fake, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_finalize_mask(fake, fake, 2, 8, 8, -1, fake, None) == _lib.E_INVALID
+    nnz, npat, nnzp = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+    assert lib.calibatt_compile_size(fake, 1, 8, 40000, 1, ctypes.byref(nnz), ctypes.byref(npat), ctypes.byref(nnzp),
+                                     fake, 1 << 20, None) == _lib.E_UNSUPPORTED
+    assert lib.calibatt_compile_size(fake, 1, 8, 8, 9, ctypes.byref(nnz), ctypes.byref(npat), ctypes.byref(nnzp),
+                                     fake, 1 << 20, None) == _lib.E_INVALID
+    assert lib.calibatt_compile(fake, 1, 8, 8, 1, 128, 128, None, fake, 1 << 20, None) == _lib.E_INVALID
+    assert lib.calibatt_selftest_wait_timeout(0, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_selftest_wait_timeout(1000, None, None) == _lib.E_INVALID
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    import block_sparse_attention_cross_b200 as cba
+    x = torch.zeros(1, 1, 128, 64)
+    with pytest.raises(ValueError):
+        cba.sparse_attn_fwd(x, x, x, None, 128)

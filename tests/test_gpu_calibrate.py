@@ -1,0 +1,130 @@
+"""GPU calibration against the oracle.
+
+Energies are floating point: compared with a tolerance.  Selection, votes and
+masks are discrete: fed the GPU's own energies, the oracle must reproduce
+them bit for bit.  End to end (oracle energies in float64), masks may differ
+only in near-tie rows, whose boundary gap is below 1e-4 of the row's largest
+energy.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_cross_b200 as cba
+from block_sparse_attention_cross_b200 import synthetic as syn
+import oracle
+
+from _util import bf16_pair, fp32_pair
+
+pytestmark = pytest.mark.gpu
+
+
+def small_inputs(n_inputs, H, grid, d, seed_base=10):
+    w = syn.Workload("calib_small", 1, H, grid, d, "bf16", 128, 0.25,
+                     {"base": seed_base, "noise_q": 11, "noise_k": 12, "v": 13})
+    out = []
+    for n in range(n_inputs):
+        q, k = syn.video_qkv(w, with_v=False, input_index=n)
+        out.append((q[0], k[0]))
+    return w, out
+
+
+@pytest.mark.parametrize("dtype,d,block", [("fp32", 64, 64), ("fp32", 128, 128), ("bf16", 128, 128), ("bf16", 64, 128)])
+def test_block_energy(dtype, d, block):
+    H = 2
+    w, inputs = small_inputs(1, H, syn.VideoGrid(2, 20, 50), d)
+    q, k = inputs[0]
+    pair = bf16_pair if dtype == "bf16" else fp32_pair
+    q64, qd = pair(q)
+    k64, kd = pair(k)
+    scale = cba.default_scale(d)
+    E = cba.block_energy(qd, kd, w.N, block, block, scale=scale).cpu().numpy().astype(np.float64)
+    Eo = oracle.block_energy(q64, k64, w.N, block, block, scale)
+    nreal = -(-w.N // block)
+    rel = np.abs(E - Eo).max()
+    assert rel <= (1e-5 if dtype == "fp32" else 5e-5), rel
+    np.testing.assert_allclose(E[:, :nreal].sum(axis=-1), 1.0, atol=1e-4)
+
+
+def test_select_vote_finalize_bit_exact():
+    rng = np.random.default_rng(4)
+    H, nqb, nkb, I = 3, 9, 37, 5
+    Es = [rng.random((H, nqb, nkb)).astype(np.float32) for _ in range(I)]
+    Es[0][0, 0, 5] = Es[0][0, 0, 6]                      # exact tie
+    Es[1][1, 2, :] = 0.25                                # all ties
+    for mode, param in ((cba.SELECT_TOPK, 0.25), (cba.SELECT_ENERGY, 0.3), (cba.SELECT_ENERGY, 0.0)):
+        votes = torch.zeros((H, nqb, nkb), dtype=torch.int32, device="cuda")
+        esum = torch.zeros((H, nqb, nkb), dtype=torch.float32, device="cuda")
+        keeps = []
+        for E in Es:
+            cba.select_vote(torch.from_numpy(E).cuda(), mode, param, votes, esum)
+            keeps.append(oracle.select_topk(E, param) if mode == cba.SELECT_TOPK else oracle.select_energy(E, param))
+        for mv in (1, 3, 5):
+            mask = cba.finalize_mask(votes, esum, mv)
+            m_o, v_o, e_o = oracle.vote(np.stack(keeps), mv, np.stack(Es))
+            assert np.array_equal(votes.cpu().numpy(), v_o)
+            assert np.array_equal(esum.cpu().numpy(), e_o)
+            assert np.array_equal(mask.cpu().numpy(), m_o)
+
+
+def near_tie_rows(E, k):
+    """Rows whose k-th and (k+1)-th energies are closer than 1e-4 of the row maximum."""
+    s = -np.sort(-E, axis=-1)
+    gap = s[..., k - 1] - s[..., k]
+    return gap < 1e-4 * s[..., 0]
+
+
+def test_calibrate_small_end_to_end():
+    H, I = 2, 4
+    w, inputs = small_inputs(I, H, syn.VideoGrid(3, 30, 52), 128)
+    nb = w.Np // 128
+    pairs = [(bf16_pair(q), bf16_pair(k)) for q, k in inputs]
+    qd = [p[0][1] for p in pairs]
+    kd = [p[1][1] for p in pairs]
+    mv = cba.min_votes_for(0.5, I)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mask, votes, esum = cba.calibrate(qd, kd, w.N, select_param=0.25, rho=0.5, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    # discrete stages on the GPU's energies: bit-exact
+    Eg = [cba.block_energy(q, k, w.N).cpu().numpy() for q, k in zip(qd, kd)]
+    keeps = [oracle.select_topk(E, 0.25) for E in Eg]
+    m_o, v_o, e_o = oracle.vote(np.stack(keeps), mv, np.stack(Eg))
+    assert np.array_equal(votes.cpu().numpy(), v_o)
+    assert np.array_equal(esum.cpu().numpy(), e_o)
+    assert np.array_equal(mask.cpu().numpy(), m_o)
+    # end to end against float64 energies: differences only in near-tie rows
+    Eo = [oracle.block_energy(p[0][0], p[1][0], w.N, 128, 128, cba.default_scale(128)) for p in pairs]
+    k = oracle.topk_count(0.25, nb)
+    keeps64 = [oracle.select_topk(E, 0.25) for E in Eo]
+    m64, _, _ = oracle.vote(np.stack(keeps64), mv, np.stack(Eo))
+    tie = np.zeros((H, nb), bool)
+    for E in Eo:
+        tie |= near_tie_rows(E, k)
+    diff_rows = (mask.cpu().numpy() != m64).any(axis=-1)
+    assert not (diff_rows & ~tie).any()
+    # the compiled calibrated mask drives the forward kernel
+    bl = cba.compile(mask)
+    assert bl.nnz == int(mask.sum().item())
+
+
+@pytest.mark.slow
+def test_calibrate_wan_config_subset():
+    # 8 calibration inputs of the Wan 480p shape; the oracle's discrete stages
+    # run on the GPU's energies for every head.
+    w = syn.WORKLOADS["wan480_25"]
+    I = 8
+    qd, kd = [], []
+    for n in range(I):
+        q, k = syn.video_qkv(w, with_v=False, input_index=n)
+        qd.append(bf16_pair(q[0])[1])
+        kd.append(bf16_pair(k[0])[1])
+        del q, k
+    mask, votes, esum = cba.calibrate(qd, kd, w.N, select_param=0.25, rho=0.5)
+    Eg = [cba.block_energy(q, k, w.N).cpu().numpy() for q, k in zip(qd, kd)]
+    keeps = [oracle.select_topk(E, 0.25) for E in Eg]
+    m_o, v_o, _ = oracle.vote(np.stack(keeps), 4, np.stack(Eg))
+    assert np.array_equal(votes.cpu().numpy(), v_o)
+    assert np.array_equal(mask.cpu().numpy(), m_o)
+    np.testing.assert_allclose(np.stack(Eg)[:, :, :, :].sum(axis=-1), 1.0, atol=2e-3)

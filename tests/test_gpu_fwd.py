@@ -1,0 +1,154 @@
+"""GPU parity of calibatt_sparse_attn_fwd against the float64 oracle.
+
+bf16 (tcgen05 tensor-core kernel): O within max-abs 2e-2 and mean-abs 2e-3,
+LSE within 1e-3.  fp32 (FFMA kernel): O within 1e-5, LSE within 1e-5.
+Small cases are compared on every row; full-size workloads on sampled query
+blocks that the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_cross_b200 as cba
+from block_sparse_attention_cross_b200 import synthetic as syn
+import oracle
+
+from _util import (BF16_MAX_ABS, BF16_MEAN_ABS, FP32_MAX_ABS, assert_close, assert_lse, bf16_pair, fp32_pair,
+                   to_np64)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_full_compare(q, k, v, mask, N, block, dtype, d, B=1, H=None, map_offset=0, lse_tol=None):
+    """Whole-tensor parity of one small case."""
+    pair = bf16_pair if dtype == "bf16" else fp32_pair
+    q64, qd = pair(q)
+    k64, kd = pair(k)
+    v64, vd = pair(v)
+    bl = cba.compile(torch.from_numpy(mask).cuda(), block_q=block, block_k=block)
+    H = q.shape[1]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = cba.default_scale(d)
+    o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, N, scale=scale, map_offset=map_offset, return_lse=True,
+                                 status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    O, L = oracle.masked_attention(q64, k64, v64, mask[map_offset:map_offset + H], N, block, block, scale)
+    if dtype == "bf16":
+        mx, mn = assert_close(to_np64(o), O, BF16_MAX_ABS, BF16_MEAN_ABS)
+        assert_lse(lse.cpu().numpy(), L, lse_tol or 1e-3)
+    else:
+        mx, mn = assert_close(to_np64(o), O, FP32_MAX_ABS)
+        assert_lse(lse.cpu().numpy(), L, lse_tol or 1e-5)
+    return mx, mn
+
+
+def test_fp32_tiny_config():
+    w = syn.WORKLOADS["tiny_fp32"]
+    q, k, v = syn.normal_qkv(w.B, w.H, w.N, w.Np, w.d, w.seeds["data"])
+    mask = syn.workload_mask(w)
+    run_full_compare(q, k, v, mask, w.N, w.block, "fp32", w.d)
+
+
+@pytest.mark.parametrize("d,block", [(128, 128), (64, 128), (128, 64)])
+def test_fp32_ragged_with_empty_rows(d, block):
+    N, Np, H = 1000, 1024, 2
+    q, k, v = syn.normal_qkv(2, H, N, Np, d, 7)
+    nb = Np // block
+    mask = (np.random.default_rng(3).random((H + 1, nb, nb)) < 0.4).astype(np.uint8)
+    mask[0, 2, :] = 0                   # empty row
+    mask[1, nb - 1, :] = 0              # empty last (padded) row
+    mask[1, 0, nb - 1] = 1              # padded key block kept
+    run_full_compare(q, k, v, mask, N, block, "fp32", d, map_offset=0)
+    run_full_compare(q, k, v, mask, N, block, "fp32", d, map_offset=1)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_small_random_masks(d):
+    N, Np, H = 1000, 1024, 3
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 11)
+    mask = (np.random.default_rng(5).random((H, 8, 8)) < 0.5).astype(np.uint8)
+    mask[0, 3, :] = 0                   # empty row
+    mask[1, :, 7] = 1                   # padded key block everywhere
+    mask[2, 7, :] = 1                   # padded query block sees all
+    run_full_compare(q, k, v, mask, N, 128, "bf16", d)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_full_mask_is_dense(d):
+    N, Np, H = 2040, 2048, 2
+    q, k, v = syn.normal_qkv(2, H, N, Np, d, 12)
+    mask = np.ones((H, 16, 16), np.uint8)
+    run_full_compare(q, k, v, mask, N, 128, "bf16", d)
+
+
+def test_bf16_structured_scores():
+    # Wan-like structured Q/K (logit std ~3) with a structured mask, 4 frames
+    w = syn.Workload("wan_small", 2, 2, syn.VideoGrid(4, 30, 52), 128, "bf16", 128, 0.3,
+                     {"base": 10, "noise_q": 11, "noise_k": 12, "v": 13, "mask": 14})
+    q, k, v = syn.video_qkv(w)
+    mask = syn.workload_mask(w)
+    run_full_compare(q, k, v, mask, w.N, 128, "bf16", 128)
+
+
+def test_bf16_deterministic():
+    N, Np, H = 1024, 1024, 2
+    q, k, v = syn.normal_qkv(1, H, N, Np, 128, 21)
+    _, qd = bf16_pair(q)
+    _, kd = bf16_pair(k)
+    _, vd = bf16_pair(v)
+    mask = (np.random.default_rng(9).random((H, 8, 8)) < 0.5).astype(np.uint8)
+    bl = cba.compile(torch.from_numpy(mask).cuda())
+    o1, l1 = cba.sparse_attn_fwd(qd, kd, vd, bl, N, return_lse=True)
+    o2, l2 = cba.sparse_attn_fwd(qd, kd, vd, bl, N, return_lse=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def sampled_parity(w, mask, qkv=None, n_samples=24, seed=0, map_offset=0):
+    """Full-size run; oracle on sampled (head, query block) pairs incl. the first and last block."""
+    q, k, v = qkv if qkv is not None else syn.video_qkv(w)
+    q64, qd = bf16_pair(q)
+    del q
+    k64, kd = bf16_pair(k)
+    del k
+    v64, vd = bf16_pair(v)
+    del v
+    bl = cba.compile(torch.from_numpy(mask).cuda())
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = cba.default_scale(w.d)
+    o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, w.N, scale=scale, map_offset=map_offset, return_lse=True,
+                                 status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rng = np.random.default_rng(seed)
+    picks = [(0, 0), (w.H - 1, w.nqb - 1)] + [(int(rng.integers(w.H)), int(rng.integers(w.nqb)))
+                                              for _ in range(n_samples - 2)]
+    errs = []
+    for h, qb in picks:
+        O, L = oracle.masked_attention_rows(q64, k64, v64, mask[map_offset:], w.N, w.block, w.block, scale, 0, h, qb)
+        rows = slice(qb * w.block, (qb + 1) * w.block)
+        got = to_np64(o[0, h, rows])
+        errs.append(np.abs(got - O))
+        assert_lse(lse[0, h, rows].cpu().numpy(), L, 1e-3)
+    err = np.concatenate([e.ravel() for e in errs])
+    assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
+    return err.max(), err.mean()
+
+
+@pytest.mark.slow
+def test_bf16_wan480_full_size_sampled():
+    w = syn.WORKLOADS["wan480_25"]
+    sampled_parity(w, syn.workload_mask(w))
+
+
+@pytest.mark.slow
+def test_bf16_wan720_full_size_sampled():
+    w = syn.WORKLOADS["wan720_20"]
+    sampled_parity(w, syn.workload_mask(w), n_samples=12)
+
+
+@pytest.mark.slow
+def test_bf16_mochi_full_size_sampled():
+    w = syn.WORKLOADS["mochi_20"]
+    sampled_parity(w, syn.workload_mask(w), n_samples=12)
