@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the calibrated block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl calibatt|reference]
+
+One step is one block-sparse attention call of the Wan-2.1-14B-shaped
+workload (21 x 30 x 52 = 32760 tokens padded to 32768, 40 heads, d = 128,
+bf16, 128 x 128 blocks, 25% of the blocks kept by a structured mask).  The
+inputs are seeded and synthetic (shared low-rank frame/row/column structure
+plus noise for Q and K, Gaussian V); they are 1.0 GB, larger than the 126 MB
+L2, and are not flushed between steps.
+
+The headline ``value`` is kept-block TFLOP/s (4 * 128 * 128 * d FLOP per
+kept block, summed over heads and ranks) with inputs resident in HBM, timed
+on the device with CUDA events over exactly K steps bracketed by barriers
+and synchronizations; the maximum over ranks is used.  ``e2e`` is the same
+metric when every step also copies Q, K, V from pinned host memory and reads
+O back.  With N > 1 ranks (torchrun, NCCL) every rank runs its own replica
+(weak scaling, no collective on the data path).
+
+``--impl reference`` times the float64 CPU oracle (the only other place that
+executes ``oracle/``) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+METRIC = "sparse attn fwd kept-block TFLOP/s, % bf16 TC peak; speedup vs full-mask"
+UNIT = "TFLOP/s"
+WORKLOAD = "wan480_25"
+KERNEL_SOURCE = ROOT / "block_sparse_attention_cross_b200" / "csrc" / "attn_tc.cu"
+TRAFFIC_FILE = ROOT / "profiles" / "traffic.json"
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["calibatt", "reference"], default="calibatt")
+    p.add_argument("--no-extras", action="store_true", help="skip the density sweep, e2e and CPU baseline")
+    p.add_argument("--heads", type=int, default=None,
+                   help="use only the first H heads (a smaller case for profiling; default: all 40)")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def physical_gpu_id(local):
+    """nvidia-smi id (index or UUID) of this rank's GPU."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def kept_flops(nnz_blocks, d, B, block=128):
+    return 4.0 * block * block * d * B * nnz_blocks
+
+
+def peaks():
+    f = ROOT / "MEASURED_PEAKS.json"
+    if f.exists():
+        p = json.loads(f.read_text())
+        return {"bf16_burst": float(p["bf16_tflops"]), "bf16_sustained": float(p.get("bf16_tflops_sustained",
+                                                                                      p["bf16_tflops"])),
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = Path(os.environ.get("TMPDIR", "/tmp")) / f"calibatt_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in self.path.read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7], "power_cap": parts[8]})
+            except ValueError:
+                continue
+        self.path.unlink(missing_ok=True)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("power_cap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def workload(heads=None):
+    import dataclasses
+    from block_sparse_attention_cross_b200 import synthetic as syn
+    w = syn.WORKLOADS[WORKLOAD]
+    return dataclasses.replace(w, H=heads) if heads else w
+
+
+def build_workload(device, heads=None, density=None):
+    import torch
+    import block_sparse_attention_cross_b200 as cba
+    from block_sparse_attention_cross_b200 import synthetic as syn
+    w = workload(heads)
+    q, k, v = syn.video_qkv(w)
+    tensors = []
+    for x in (q, k, v):
+        bits = syn.f32_to_bf16_bits(x)
+        tensors.append(torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16))
+    del q, k, v
+    mask = torch.from_numpy(syn.workload_mask(w, density=density)).to(device)
+    bl = cba.compile(mask)
+    return w, tensors, bl
+
+
+def sampled_blocks(w, n_heads, per_head, seed=123):
+    rng = np.random.default_rng(seed)
+    heads = sorted(rng.choice(w.H, size=min(n_heads, w.H), replace=False).tolist())
+    picks = []
+    for h in heads:
+        rest = [int(x) for x in rng.permutation(np.arange(1, w.nqb - 1))]
+        picks += [(h, qb) for qb in ([0, w.nqb - 1] + rest)[:per_head]]
+    return picks
+
+
+def run_oracle_sample(w, qkv_np, mask, picks, scale):
+    """Times the float64 oracle on (head, query block) picks; returns (seconds, kept blocks)."""
+    import oracle
+    q, k, v = qkv_np
+    kept = 0
+    t0 = time.perf_counter()
+    cache = {}
+    for h, qb in picks:
+        if h not in cache:
+            cache.clear()
+            cache[h] = tuple(x[:, h:h + 1].astype(np.float64) for x in (q, k, v))
+        qh, kh, vh = cache[h]
+        oracle.masked_attention_rows(qh, kh, vh, mask[h:h + 1], w.N, w.block, w.block, scale, 0, 0, qb)
+        kept += int(mask[h, qb].sum())
+    return time.perf_counter() - t0, kept
+
+
+def oracle_inputs(w):
+    from block_sparse_attention_cross_b200 import synthetic as syn
+    q, k, v = syn.video_qkv(w)
+    out = tuple(syn.round_to_bf16(x) for x in (q, k, v))
+    mask = syn.workload_mask(w)
+    return out, mask
+
+
+def cpu_baseline(w, target_seconds=15.0):
+    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1)."""
+    import block_sparse_attention_cross_b200 as cba
+    qkv, mask = oracle_inputs(w)
+    scale = cba.default_scale(w.d)
+    probe = sampled_blocks(w, 1, 4, seed=7)
+    t, kept = run_oracle_sample(w, qkv, mask, probe, scale)
+    per_block = t / max(1, len(probe))
+    per_head = max(2, min(w.nqb, int(target_seconds / max(per_block, 1e-6) / 8)))
+    picks = sampled_blocks(w, 8, per_head)
+    t, kept = run_oracle_sample(w, qkv, mask, picks, scale)
+    return {"value": kept_flops(kept, w.d, 1) / t / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{len(picks)} (head, query-block) pairs of the {WORKLOAD} call ({kept} kept blocks, "
+                      f"incl. first and last query block), float64 numpy on {cpu_model()}; {t:.1f} s",
+            "seconds": t}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def time_calls(fn, steps, warmup, torch, dist=None):
+    for _ in range(warmup):
+        fn()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(s)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(s)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[-1]), per
+
+
+def kernel_traffic():
+    """DRAM bytes per launch from the committed ncu capture, if the kernel source is unchanged."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    rec = json.loads(TRAFFIC_FILE.read_text())
+    sha = hashlib.sha256(KERNEL_SOURCE.read_bytes()).hexdigest()
+    if rec.get("kernel_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def main_calibatt(args):
+    import torch
+    import block_sparse_attention_cross_b200 as cba
+    world, rank, local = dist_env()
+    dist = None
+    if world > 1:
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w, (q, k, v), bl = build_workload(dev, args.heads)
+    out = torch.empty_like(q)
+    pk = peaks()
+    flops_step = kept_flops(bl.nnz, w.d, w.B)
+
+    def step():
+        cba.sparse_attn_fwd(q, k, v, bl, w.N, out=out)
+
+    warm = max(3, args.warmup)
+    launches0 = cba.launch_count()
+    clocks = ClockSampler(physical_gpu_id(local))
+    for _ in range(warm):
+        step()
+    launches_warm = cba.launch_count()
+    clocks.start()
+    total_ms, per = time_calls(step, args.steps, 0, torch, dist)
+    clk = clocks.stop()
+    launches = cba.launch_count() - launches_warm
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t_max = float(t.item())
+    value = world * flops_step * args.steps / (t_max / 1e3) / 1e12
+    ms_step = t_max / args.steps
+    per_launch_ms = statistics.mean(per)
+    achieved = flops_step / (per_launch_ms / 1e3) / 1e12
+
+    extras = {}
+    if not args.no_extras:
+        # full-mask run of the same kernel (same inputs) and a density sweep
+        full = cba.compile(torch.ones((w.H, w.nqb, w.nqb), dtype=torch.uint8, device=dev))
+        tf, _ = time_calls(lambda: cba.sparse_attn_fwd(q, k, v, full, w.N, out=out), 20, 3, torch)
+        t_full = tf / 20
+        extras["speedup_vs_full_mask"] = t_full / ms_step
+        extras["full_mask_ms"] = t_full
+        extras["full_mask_tflops"] = kept_flops(full.nnz, w.d, w.B) / (t_full / 1e3) / 1e12
+        sweep = []
+        for dens in (1.0, 0.8, 0.6, 0.4, 0.25, 0.2, 0.1):
+            from block_sparse_attention_cross_b200 import synthetic as syn
+            m = torch.from_numpy(syn.workload_mask(w, density=dens)).to(dev) if dens < 1.0 else None
+            b = cba.compile(m) if m is not None else full
+            td, _ = time_calls(lambda: cba.sparse_attn_fwd(q, k, v, b, w.N, out=out), 20, 3, torch)
+            sweep.append({"density": round(b.density, 4), "ms": round(td / 20, 4),
+                          "kept_tflops": round(kept_flops(b.nnz, w.d, w.B) / (td / 20 / 1e3) / 1e12, 1)})
+        extras["density_sweep"] = sweep
+        # end to end through the public API with host buffers
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty_like(hq).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            cba.sparse_attn_fwd(q, k, v, bl, w.N, out=out)
+            ho.copy_(out, non_blocking=True)
+
+        te, _ = time_calls(e2e_step, 10, 3, torch, dist)
+        te_t = torch.tensor([te], device=dev, dtype=torch.float64)
+        if dist is not None:
+            dist.all_reduce(te_t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te_t.item()) / 10
+        extras["e2e"] = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                         "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
+                         "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": warm, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: Wan-2.1-14B-shaped attention call, 21x30x52 = 32760 tokens "
+                                   f"(padded {w.Np}), {w.H} heads, d={w.d}, bf16, 128x128 blocks, "
+                                   f"{100 * bl.density:.1f}% of blocks kept (structured mask)",
+                       "B": w.B, "H": w.H, "N": w.N, "Np": w.Np, "d": w.d, "block": w.block,
+                       "kept_blocks": bl.nnz, "density": round(bl.density, 6),
+                       "l2": "inputs 1.0 GB > 126 MB L2; no flush between steps",
+                       "parallelism": f"replicas x{world} (head-sharded work is independent)"},
+            "pct_bf16_peak_burst": round(100 * value / world / pk["bf16_burst"], 2),
+            "pct_bf16_peak_sustained": round(100 * value / world / pk["bf16_sustained"], 2),
+            "dense_equiv_tflops": round(world * 4.0 * w.N * w.N * w.d * w.H * w.B / (ms_step / 1e3) / 1e12, 2),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_sustained"],
+                         "unit": UNIT, "frac": round(achieved / pk["bf16_sustained"], 4),
+                         "traffic": kernel_traffic(),
+                         "kernel": "k_attn_tc<128, MODE_FWD>",
+                         "peak_kind": f"bf16_tflops_sustained ({pk['source']}); burst {pk['bf16_burst']}",
+                         "algorithmic_flops_per_launch": flops_step},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        line.update({k2: v2 for k2, v2 in extras.items() if k2 != "e2e"})
+        if "e2e" in extras:
+            line["e2e"] = extras["e2e"]
+        if world == 1 and not args.no_extras:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def main_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import block_sparse_attention_cross_b200 as cba  # noqa: F401  (scale helper only)
+    w = workload(args.heads)
+    qkv, mask = oracle_inputs(w)
+    scale = cba.default_scale(w.d)
+    steps, warm = args.steps, max(3, args.warmup)
+    probe = sampled_blocks(w, 1, 2, seed=3)
+    t_probe, _ = run_oracle_sample(w, qkv, mask, probe, scale)
+    per_block = t_probe / len(probe)
+    budget = 150.0  # seconds for warmup + timed steps
+    blocks_per_step = max(1, int(budget / (steps + warm) / max(per_block, 1e-6)))
+    rng = np.random.default_rng(11)
+
+    def one_step():
+        picks = [(int(rng.integers(w.H)), int(rng.integers(w.nqb))) for _ in range(blocks_per_step)]
+        return run_oracle_sample(w, qkv, mask, picks, scale)
+
+    for _ in range(warm):
+        one_step()
+    tot_t, tot_kept = 0.0, 0
+    for _ in range(steps):
+        t, kept = one_step()
+        tot_t += t
+        tot_kept += kept
+    value = kept_flops(tot_kept, w.d, 1) / tot_t / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
+        "ms_per_step": 1e3 * tot_t / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{WORKLOAD} (sampled query blocks per step)", "B": w.B, "H": w.H, "N": w.N,
+                   "Np": w.Np, "d": w.d, "block": w.block, "density": w.density,
+                   "blocks_per_step": blocks_per_step},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"{blocks_per_step} random (head, query-block) pairs per step, float64 numpy "
+                                   f"on {cpu_model()}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    sys.path.insert(0, str(ROOT))
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_calibatt(args)
+
+
+if __name__ == "__main__":
+    main()
