@@ -27,7 +27,7 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
                    CalibattError, check, load)
 
 __all__ = [
-    "BlockList", "sparse_attn_fwd", "block_energy", "select_vote", "finalize_mask", "calibrate",
+    "BlockList", "sparse_attn_fwd", "block_energy", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -169,6 +169,26 @@ def block_energy(q, k, N, block_q=128, block_k=128, scale=None, status=None, wor
     with torch.cuda.device(q.device):
         check(load().calibatt_block_energy(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q, block_k,
                                            scale, _ptr(E), _ptr(ws), ws.numel(), _ptr(status), _stream(q.device)))
+    return E
+
+
+def block_energy_noalloc(q, k, N, block_q=128, block_k=128, scale=None, status=None, out=None):
+    """Block energies like :func:`block_energy`, without any device allocation by the library.
+
+    For callers that cannot hand the library a workspace: the per-row scratch
+    lives in a fixed 16 MiB array inside the library (H * Np <= 4 Mi rows).
+    Calls that overlap on the GPU share that array and must not be issued.
+    Pass ``out`` ([H, nqb, nkb] float32) to avoid the one allocation this
+    wrapper would otherwise make for the result.
+    """
+    _need_cuda(q, k)
+    H, Np, d = q.shape
+    scale = default_scale(d) if scale is None else float(scale)
+    E = torch.empty((H, Np // block_q, Np // block_k), device=q.device, dtype=torch.float32) if out is None else out
+    _need_cuda(E, status)
+    with torch.cuda.device(q.device):
+        check(load().calibatt_block_energy_noalloc(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q,
+                                                   block_k, scale, _ptr(E), _ptr(status), _stream(q.device)))
     return E
 
 

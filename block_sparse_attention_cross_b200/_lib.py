@@ -41,6 +41,8 @@ EXPORTS = {
                                          c_int, c_int, c_int, c_float, c_void_p, c_int, c_void_p, c_void_p]),
     "calibatt_block_energy": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "calibatt_block_energy_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                              c_float, c_void_p, c_void_p, c_void_p]),
     "calibatt_calibrate_workspace_size": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, POINTER(c_size_t)]),
     "calibatt_select_vote": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_double, c_void_p, c_void_p, c_void_p]),
     "calibatt_finalize_mask": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),

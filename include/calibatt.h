@@ -229,6 +229,33 @@ int calibatt_compile(const uint8_t* masks, int n_maps, int nqb, int nkb, int ded
                      void* workspace, size_t workspace_bytes, calibatt_stream_t stream);
 
 /*
+ * calibatt_block_energy_noalloc -- calibatt_block_energy for callers that
+ * cannot allocate device memory.
+ *
+ * The paper has no counterpart: this is a deployment variant.  Some callers
+ * hold only their input and output buffers -- a plugin whose host engine
+ * hands it no workspace, or a service that reserved the GPU's memory for its
+ * own pool at start-up and allows no allocation afterwards -- so they cannot
+ * supply the per-row scratch that calibatt_block_energy takes as workspace.
+ * This entry point keeps that scratch in a fixed array inside the library's
+ * device memory (16 MiB, held on every GPU that loads the library until the
+ * process exits) and allocates nothing.  Same arguments, result and
+ * supported shapes as calibatt_block_energy, minus the workspace.
+ *
+ *  - H * Np must be <= 4 194 304 (the array holds one float per query row);
+ *    larger calls return CALIBATT_E_WORKSPACE and launch nothing.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - Every call shares the one array.  Calls on one stream are ordered;
+ *    calls that overlap on the GPU (other streams, other threads on the same
+ *    device) race on the scratch and must not be issued.
+ */
+int calibatt_block_energy_noalloc(const void* q, const void* k, int H, int N, int Np, int d, int dtype,
+                                  int block_q, int block_k, float scale, float* energy_out,
+                                  int32_t* dev_status, calibatt_stream_t stream);
+
+/*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the
  * bounded wait every kernel here uses, on a barrier that nothing completes.
  * After `limit_ns` it gives up and writes CALIBATT_E_TIMEOUT to dev_status.
