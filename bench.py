@@ -41,7 +41,7 @@ ROOT = Path(__file__).resolve().parent
 METRIC = "sparse attn fwd kept-block TFLOP/s, % bf16 TC peak; speedup vs full-mask"
 UNIT = "TFLOP/s"
 WORKLOAD = "wan480_25"
-KERNEL_SOURCE = ROOT / "block_sparse_attention_cross_b200" / "csrc" / "attn_tc.cu"
+KERNEL_SOURCE = ROOT / "block_sparse_attention_cross_b200" / "csrc" / "attn_fwd.cu"
 TRAFFIC_FILE = ROOT / "profiles" / "traffic.json"
 
 
@@ -371,7 +371,7 @@ def main_calibatt(args):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_sustained"],
                          "unit": UNIT, "frac": round(achieved / pk["bf16_sustained"], 4),
                          "traffic": kernel_traffic(),
-                         "kernel": "k_attn_tc<128, MODE_FWD>",
+                         "kernel": "k_attn_fwd<128>",
                          "peak_kind": f"bf16_tflops_sustained ({pk['source']}); burst {pk['bf16_burst']}",
                          "algorithmic_flops_per_launch": flops_step},
             "gpu_launches": int(launches),

@@ -1,0 +1,566 @@
+// attn_fwd.cu -- persistent block-sparse flash-attention forward for sm_100a.
+//
+// CalibAtt (arXiv 2603.05503, paper page, Abstract and Figure 5(b) top): the
+// kept blocks of the calibrated mask are computed densely and the others are
+// skipped.  Each query tile (128 rows of one batch/head) walks its compiled
+// kept-block list; only the kept K/V tiles are loaded (TMA) and multiplied
+// (tcgen05), so a skipped block costs neither bytes nor FLOPs.
+//
+// Persistent CTA (one per SM), 12 warps, two independent query-tile "slots":
+//   warps 0-3   softmax warpgroup of slot 0 (thread t owns row t = TMEM lane t)
+//   warps 4-7   softmax warpgroup of slot 1
+//   warp 8      TMA producer: Q tile per slot, K and V tiles of the kept blocks
+//               into one shared ring, in exactly the order the MMA warp uses them
+//   warp 9      TMEM allocator and MMA issuer
+//   warps 10-11 idle (they complete the control warpgroup)
+// The block is launched with 168 registers per thread.  Inside its own branch
+// the control warpgroup lowers its limit to 88 and the softmax warpgroups
+// raise theirs to 208, which holds a full 128-column score row in registers:
+// 2 * 128 * 208 + 128 * 88 = 384 * 168.
+// The two slots have their own kept-block lists; while one slot's softmax
+// runs, the tensor core works on the other slot's QK^T and PV, so neither
+// waits for the other.  Per slot and block j the MMA issue order is
+// PV(j-1), S(j): S(j) overwrites the TMEM columns holding P(j-1), which the
+// in-order tensor pipe has already consumed.
+//
+// TMEM (512 columns): slot s uses [256 s, 256 s + 128) for S, overwritten in
+// place by P as bf16 pairs (the A operand of the PV MMA), and
+// [256 s + 128, 256 s + 128 + d) for the O accumulator.
+// Softmax: exp2 on the scaled scores; the running max is only raised (and O
+// rescaled in TMEM) when it grows by more than 8 (log2 units), which keeps
+// every P value <= 256 and O / l exact.
+// Every wait is bounded; on expiry the CTA reports CALIBATT_E_TIMEOUT, drains
+// its own copies and MMAs, frees TMEM and exits.
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace calibatt {
+namespace {
+
+constexpr int TILE = 128;
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 208;
+constexpr uint32_t kControlRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs, "register split");
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdLayout {
+  static constexpr uint32_t BOX_BYTES = TILE * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
+  static constexpr uint32_t TILE_BYTES = TILE * D * 2;
+  static constexpr int RING = (D == 128) ? 5 : 10;
+  static constexpr uint32_t OFF_Q = 0;                   // 2 slots
+  static constexpr uint32_t OFF_RING = 2 * TILE_BYTES;
+  static constexpr uint32_t OFF_CTRL = OFF_RING + RING * TILE_BYTES;
+  static constexpr uint32_t CTRL_BYTES = 1024;
+  static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
+};
+
+template <int RING>
+struct FwdCtrl {
+  uint64_t ring_full[RING], ring_empty[RING];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full[2], o_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
+__device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
+
+struct TileList {
+  int bh, h, qb;
+  int n;      // kept blocks (0 for an empty or rejected list)
+  int base;   // first kept block
+  int p0;     // start of the pattern in pat_off
+};
+
+// Reads and checks the kept-block list of work tile t.  Warp-collective: every
+// lane returns the same result, and every role evaluates the same data, so
+// all roles agree on n.
+__device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool report) {
+  TileList tl;
+  tl.bh = t / a.nqb;
+  tl.qb = t - tl.bh * a.nqb;
+  tl.h = tl.bh % a.H;
+  const long long r = static_cast<long long>(a.map_offset + tl.h) * a.nqb + tl.qb;
+  tl.base = a.row_base[r];
+  const int pat = a.row_pat[r];
+  bool bad = false;
+  int p0 = 0, p1 = 0;
+  if (pat < 0 || pat >= a.n_pat) {
+    bad = true;
+  } else {
+    p0 = a.pat_ptr[pat];
+    p1 = a.pat_ptr[pat + 1];
+    if (p0 < 0 || p1 < p0 || p1 > a.nnz_pat || p1 - p0 > a.nkb) bad = true;
+  }
+  const int n = bad ? 0 : p1 - p0;
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < n; i += 32) {
+    const int off = a.pat_off[p0 + i];
+    const int kb = tl.base + off;
+    bool ok = kb >= 0 && kb < a.nkb;
+    if (i > 0) ok = ok && off > a.pat_off[p0 + i - 1];
+    bad |= !ok;
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad && report && lane == 0) report_status(a.status, CALIBATT_E_CORRUPT);
+  tl.n = bad ? 0 : n;
+  tl.p0 = p0;
+  return tl;
+}
+
+// Static schedule shared by the producer and the MMA warp.  Slot s of CTA c
+// takes work tiles c + s*G, c + s*G + 2G, ... (G = gridDim.x), skipping
+// tiles with empty lists.  A step of a slot is "PV of the previous block (if
+// any), then QK^T of the next block (if any)".
+struct SlotSched {
+  int t, n, base, p0, bh, j, pv;
+  bool done;
+};
+
+__device__ __forceinline__ void sched_next_tile(const TcArgs& a, SlotSched& st, int T, int stride) {
+  while (st.t < T) {
+    const TileList tl = tile_list(a, st.t, false);
+    if (tl.n > 0) {
+      st.n = tl.n;
+      st.base = tl.base;
+      st.p0 = tl.p0;
+      st.bh = tl.bh;
+      st.j = 0;
+      st.pv = -1;
+      return;
+    }
+    st.t += stride;
+  }
+  st.done = true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  using L = FwdLayout<D>;
+  constexpr int R = L::RING;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  FwdCtrl<R>* c = reinterpret_cast<FwdCtrl<R>*>(smem + L::OFF_CTRL);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int G = gridDim.x;
+  const int T = a.B * a.H * a.nqb;
+
+  if (tid == 0) {
+    for (int e = 0; e < R; ++e) {
+      mbar_init(&c->ring_full[e], 1);
+      mbar_init(&c->ring_empty[e], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&c->q_full[s], 1);
+      mbar_init(&c->q_empty[s], 1);
+      mbar_init(&c->s_full[s], 1);
+      mbar_init(&c->p_full[s], 128);
+      mbar_init(&c->o_full[s], 1);
+      mbar_init(&c->o_free[s], 128);
+    }
+    mbar_init(&c->drain, 1);
+    c->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&c->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c->tmem_base;
+
+  if (warp >= 8) regs_dec<kControlRegs>();
+  if (warp == kProducerWarp) {
+    // ===================== TMA producer =======================================
+    SlotSched st[2];
+    for (int s = 0; s < 2; ++s) {
+      st[s].t = blockIdx.x + s * G;
+      st[s].done = false;
+      sched_next_tile(a, st[s], T, 2 * G);
+    }
+    uint32_t g = 0;         // ring fills issued
+    int qfills[2] = {0, 0};
+    bool ok = true;
+    const uint64_t pol = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    while (ok && !(st[0].done && st[1].done)) {
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (!ok) break;
+        SlotSched& q = st[s];
+        if (q.done) continue;
+        if (q.pv >= 0) {
+          const int kb = q.base + a.pat_off[q.p0 + q.pv];
+          const int row = q.bh * a.Np + kb * TILE;
+          const int e = g % R;
+          ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
+          if (ok) {
+            mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, &tmV, x * 64, row,
+                            &c->ring_full[e], pol);
+          }
+          if (!ok) break;
+          ++g;
+          q.pv = -1;
+          if (q.j == q.n) {
+            q.t += 2 * G;
+            sched_next_tile(a, q, T, 2 * G);
+            if (q.done) continue;
+          }
+        }
+        const int j = q.j;
+        if (j == 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty[s], (qfills[s] & 1) ^ 1, &c->abort, a.spin_ns));
+          if (ok) {
+            const int qrow = q.bh * a.Np + (q.t % a.nqb) * TILE;
+            mbar_arrive_expect_tx_w(&c->q_full[s], L::TILE_BYTES);
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x)
+              tma_load_2d_w(smem + L::OFF_Q + s * L::TILE_BYTES + x * L::BOX_BYTES, &tmQ, x * 64, qrow,
+                            &c->q_full[s], pol_q);
+          }
+          if (!ok) break;
+          ++qfills[s];
+        }
+        const int kb = q.base + a.pat_off[q.p0 + j];
+        const int row = q.bh * a.Np + kb * TILE;
+        const int e = g % R;
+        ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
+        if (ok) {
+          mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
+#pragma unroll
+          for (int x = 0; x < D / 64; ++x)
+            tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, &tmK, x * 64, row,
+                          &c->ring_full[e], pol);
+        }
+        if (!ok) break;
+        ++g;
+        q.pv = j;
+        q.j = j + 1;
+      }
+    }
+    if (lane == 0) {
+      if (!ok) {
+        c->abort = 1;
+        report_status(a.status, CALIBATT_E_TIMEOUT);
+      }
+      // Drain: every copy issued must have landed before the CTA may exit.
+      for (int e = 0; e < R; ++e) {
+        const uint32_t fills = (g > static_cast<uint32_t>(e)) ? (g - 1 - e) / R + 1 : 0;
+        if (fills > 0) mbar_wait(&c->ring_full[e], (fills - 1) & 1, nullptr, a.spin_ns);
+      }
+      for (int s = 0; s < 2; ++s)
+        if (qfills[s] > 0) mbar_wait(&c->q_full[s], (qfills[s] - 1) & 1, nullptr, a.spin_ns);
+    }
+  } else if (warp == kMmaWarp) {
+    // ===================== MMA issuer =========================================
+    SlotSched st[2];
+    for (int s = 0; s < 2; ++s) {
+      st[s].t = blockIdx.x + s * G;
+      st[s].done = false;
+      sched_next_tile(a, st[s], T, 2 * G);
+    }
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false);
+    constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
+    const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+    const uint32_t sRing = smem_u32(smem + L::OFF_RING);
+    uint32_t g = 0;
+    int tiles[2] = {0, 0};   // tiles started per slot
+    int pvs[2] = {0, 0};     // PV MMAs issued per slot
+    bool ok = true;
+    while (ok && !(st[0].done && st[1].done)) {
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        if (!ok) break;
+        SlotSched& q = st[s];
+        if (q.done) continue;
+        const uint32_t tS = tmem + s * 256;
+        const uint32_t tO = tS + 128;
+        if (q.pv >= 0) {
+          const int e = g % R;
+          ok = mbar_wait(&c->p_full[s], pvs[s] & 1, &c->abort, a.spin_ns) &&
+               mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns) &&
+               (q.pv > 0 || mbar_wait(&c->o_free[s], ((tiles[s] - 1) & 1) ^ 1, &c->abort, a.spin_ns));
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t sV = sRing + e * L::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(sV + kk * 2048, L::BOX_BYTES, 1024);
+              mma_bf16_ts_w(tO, tS + kk * 8, bd, IDESC_O, (q.pv > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_w(&c->ring_empty[e]);
+            if (q.pv == q.n - 1) mma_commit_w(&c->o_full[s]);
+          }
+          if (!ok) break;
+          ++g;
+          ++pvs[s];
+          q.pv = -1;
+          if (q.j == q.n) {
+            q.t += 2 * G;
+            sched_next_tile(a, q, T, 2 * G);
+            if (q.done) continue;
+          }
+        }
+        const int j = q.j;
+        const int e = g % R;
+        if (j == 0) ++tiles[s];
+        ok = (j > 0 || mbar_wait(&c->q_full[s], (tiles[s] - 1) & 1, &c->abort, a.spin_ns)) &&
+             mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t sQs = sQ + s * L::TILE_BYTES;
+          const uint32_t sK = sRing + e * L::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sQs + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+            mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          mma_commit_w(&c->s_full[s]);
+          mma_commit_w(&c->ring_empty[e]);
+          if (j == q.n - 1) mma_commit_w(&c->q_empty[s]);
+        }
+        if (!ok) break;
+        ++g;
+        q.pv = j;
+        q.j = j + 1;
+      }
+    }
+    if (!ok && lane == 0) {
+      c->abort = 1;
+      report_status(a.status, CALIBATT_E_TIMEOUT);
+    }
+    __syncwarp();
+    mma_commit_w(&c->drain);
+    mbar_wait(&c->drain, 0, nullptr, a.spin_ns);
+  } else if (warp < 8) {
+    // ===================== softmax warpgroups =================================
+    regs_inc<kSoftmaxRegs>();
+    const int s = warp >> 2;                  // slot
+    const int w = warp & 3;                   // TMEM lane quarter
+    const int row = w * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(w * 32) << 16) + s * 256;
+    const float c2 = a.scale_log2;
+    int sc = 0;      // S tiles consumed by this slot
+    int tiles = 0;   // non-empty tiles finished by this slot
+    bool ok = true;
+    for (int t = blockIdx.x + s * G; ok && t < T; t += 2 * G) {
+      const TileList tl = tile_list(a, t, true);
+      const int grow = tl.qb * TILE + row;
+      const size_t orow_idx = static_cast<size_t>(tl.bh) * a.Np + grow;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D;
+      if (tl.n == 0) {
+        uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = z;
+        if (a.lse != nullptr) a.lse[orow_idx] = -INFINITY;
+        continue;
+      }
+      const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
+      const int valid_last = (kb_last == a.nkb - 1) ? (a.N - kb_last * TILE) : TILE;
+      float m = -INFINITY;
+      float l = 0.f;
+      for (int j = 0; j < tl.n; ++j) {
+        ok = mbar_wait(&c->s_full[s], sc & 1, &c->abort, a.spin_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++sc;
+        tc_fence_after();
+        uint32_t r[TILE];
+#pragma unroll
+        for (int q4 = 0; q4 < TILE / 32; ++q4)
+          tmem_ld32(t_lane + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
+        tmem_ld_wait();
+        reg_fence(r);
+        if (j == tl.n - 1 && valid_last < TILE) {
+          // Key columns past the sequence end exist only in the last block.
+#pragma unroll
+          for (int i = 0; i < TILE; ++i)
+            if (i >= valid_last) r[i] = f2u(-INFINITY);
+        }
+        float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
+#pragma unroll
+        for (int i = 4; i < TILE; i += 8) {
+          mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
+          mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
+          mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
+          mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
+        }
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+        const float m_cand = mx * c2;
+        float alpha = 1.f;
+        if (m_cand > m + kRescaleThreshold) {   // also true for the first block (m = -inf)
+          alpha = ex2_approx(m - m_cand);
+          m = m_cand;
+        }
+        // p = 2^(s c2 - m) two columns at a time; 3 of every 8 column pairs use
+        // the FMA-pipe polynomial, the rest the MUFU unit.  P (bf16 pairs)
+        // overwrites the first 64 columns of this slot's S region, 16
+        // columns (32 probabilities) per store.
+        const uint64_t c2x2 = f2pack(c2, c2);
+        const uint64_t negm = f2pack(-m, -m);
+        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+        for (int c16 = 0; c16 < TILE / 32; ++c16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c16 * 32 + 2 * i;
+            const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
+            uint64_t pv;
+            if ((i & 7) >= 5) {
+              pv = exp2_poly2(x);
+            } else {
+              float xl, xh;
+              f2unpack(x, xl, xh);
+              pv = f2pack(ex2_approx(xl), ex2_approx(xh));
+            }
+            if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
+            float pl, ph;
+            f2unpack(pv, pl, ph);
+            pk[i] = pack_bf16x2(pl, ph);
+          }
+          tmem_st16(t_lane + c16 * 16, pk);
+        }
+        float a0, a1, b0, b1;
+        f2unpack(acc0, a0, a1);
+        f2unpack(acc1, b0, b1);
+        const float rs = (a0 + a1) + (b0 + b1);
+        l = l * alpha + rs;
+        // O holds PV(0..j-1) complete: the commit that signalled S(j) covers
+        // every MMA issued before it.
+        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+          for (int q4 = 0; q4 < D / 32; ++q4) {
+            uint32_t r[32];
+            tmem_ld32(t_lane + 128 + q4 * 32, r);
+            tmem_ld_wait();
+            reg_fence(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = f2u(u2f(r[i]) * alpha);
+            tmem_st32(t_lane + 128 + q4 * 32, r);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&c->p_full[s]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l, LSE -------------------------------------------
+      ok = mbar_wait(&c->o_full[s], tiles & 1, &c->abort, a.spin_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ++tiles;
+      tc_fence_after();
+      const bool pad_row = grow >= a.N;
+      const float inv_l = pad_row ? 0.f : 1.f / l;
+#pragma unroll
+      for (int q4 = 0; q4 < D / 32; ++q4) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + 128 + q4 * 32, r);
+        tmem_ld_wait();
+        reg_fence(r);
+        uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 pk;
+          pk.x = pack_bf16x2(u2f(r[8 * v4 + 0]) * inv_l, u2f(r[8 * v4 + 1]) * inv_l);
+          pk.y = pack_bf16x2(u2f(r[8 * v4 + 2]) * inv_l, u2f(r[8 * v4 + 3]) * inv_l);
+          pk.z = pack_bf16x2(u2f(r[8 * v4 + 4]) * inv_l, u2f(r[8 * v4 + 5]) * inv_l);
+          pk.w = pack_bf16x2(u2f(r[8 * v4 + 6]) * inv_l, u2f(r[8 * v4 + 7]) * inv_l);
+          dst[v4] = pk;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&c->o_free[s]);
+      if (a.lse != nullptr) a.lse[orow_idx] = pad_row ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+    }
+    if (!ok) {
+      c->abort = 1;
+      report_status(a.status, CALIBATT_E_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+int g_num_sms = 0;
+
+template <int D>
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
+               cudaStream_t s) {
+  auto kern = k_attn_fwd<D>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<D>::SMEM_BYTES) !=
+        cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(k_attn_fwd)");
+    configured = true;
+  }
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return check_launch("cudaFuncGetAttributes(k_attn_fwd)");
+    launch_regs = fa.numRegs;
+  }
+  // The register re-split inside the kernel is sized for exactly kLaunchRegs
+  // per thread at launch; refuse to launch a build with any other count.
+  if (launch_regs != kLaunchRegs)
+    return set_error(CALIBATT_E_UNSUPPORTED, "k_attn_fwd was built with %d registers per thread, expected %d",
+                     launch_regs, kLaunchRegs);
+  if (g_num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return check_launch("cudaDeviceGetAttribute(SM count)");
+  }
+  const long long T = static_cast<long long>(a.B) * a.H * a.nqb;
+  const int grid = static_cast<int>(std::min<long long>(g_num_sms, (T + 1) / 2));
+  kern<<<grid, kThreads, FwdLayout<D>::SMEM_BYTES, s>>>(tq, tk, tv, a);
+  count_launch();
+  return check_launch("k_attn_fwd");
+}
+
+}  // namespace
+
+int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcArgs& a, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(a.B) * a.H * a.Np;
+  int rc;
+  if ((rc = make_tmap_bf16(&tq, q, rows, d)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, rows, d)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, rows, d)) != CALIBATT_OK) return rc;
+  if (d == 128) return launch_fwd<128>(tq, tk, tv, a, s);
+  return launch_fwd<64>(tq, tk, tv, a, s);
+}
+
+}  // namespace calibatt

@@ -152,3 +152,20 @@ def test_bf16_wan720_full_size_sampled():
 def test_bf16_mochi_full_size_sampled():
     w = syn.WORKLOADS["mochi_20"]
     sampled_parity(w, syn.workload_mask(w), n_samples=12)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_persistent_schedule_ragged_lists(d):
+    # Many work tiles per CTA slot, lists from 0 to all 64 blocks, empty rows
+    # interleaved, a batch of 2 and a ragged sequence tail.
+    B, H, N, Np = 2, 5, 8000, 8064
+    nb = Np // 128
+    q, k, v = syn.normal_qkv(B, H, N, Np, d, 31)
+    rng = np.random.default_rng(8)
+    mask = np.zeros((H, nb, nb), np.uint8)
+    for h in range(H):
+        for qb in range(nb):
+            cnt = int(rng.choice([0, 1, 2, 5, 17, 40, nb]))
+            if cnt:
+                mask[h, qb, rng.choice(nb, size=cnt, replace=False)] = 1
+    run_full_compare(q, k, v, mask, N, 128, "bf16", d)
