@@ -49,6 +49,10 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Column pairs i with (i % 8) >= kPolyFrom evaluate exp2 with the FMA-pipe
+// polynomial instead of MUFU.  Measured on B200 at this instruction mix the
+// MUFU unit is not the limiter, so the polynomial is off (8).
+constexpr int kPolyFrom = 8;
 
 template <int D>
 struct FwdLayout {
@@ -308,11 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) {
             tc_fence_after();
             const uint32_t sV = sRing + e * L::TILE_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < TILE / 16; ++kk) {
-              const uint64_t bd = sdesc_sw128(sV + kk * 2048, L::BOX_BYTES, 1024);
-              mma_bf16_ts_w(tO, tS + kk * 8, bd, IDESC_O, (q.pv > 0 || kk > 0) ? 1u : 0u);
-            }
+            mma_ts_k128_w(tO, tS, sdesc_sw128(sV, L::BOX_BYTES, 1024), IDESC_O, q.pv > 0 ? 1u : 0u);
             mma_commit_w(&c->ring_empty[e]);
             if (q.pv == q.n - 1) mma_commit_w(&c->o_full[s]);
           }
@@ -336,11 +336,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sQs = sQ + s * L::TILE_BYTES;
           const uint32_t sK = sRing + e * L::TILE_BYTES;
+          if (D == 128) {
+            mma_ss_k128_w(tS, sdesc_sw128(sQs, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::BOX_BYTES >> 4);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sQs + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
-            mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(sQs + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+              mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+            }
           }
           mma_commit_w(&c->s_full[s]);
           mma_commit_w(&c->ring_empty[e]);
@@ -419,8 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           alpha = ex2_approx(m - m_cand);
           m = m_cand;
         }
-        // p = 2^(s c2 - m) two columns at a time; 3 of every 8 column pairs use
-        // the FMA-pipe polynomial, the rest the MUFU unit.  P (bf16 pairs)
+        // p = 2^(s c2 - m) two columns at a time (pairs selected by kPolyFrom
+        // use the FMA-pipe polynomial, the rest the MUFU unit).  P (bf16 pairs)
         // overwrites the first 64 columns of this slot's S region, 16
         // columns (32 probabilities) per store.
         const uint64_t c2x2 = f2pack(c2, c2);
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int e = c16 * 32 + 2 * i;
             const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
             uint64_t pv;
-            if ((i & 7) >= 5) {
+            if ((i & 7) >= kPolyFrom) {
               pv = exp2_poly2(x);
             } else {
               float xl, xh;

@@ -233,6 +233,63 @@ __device__ __forceinline__ void tma_load_2d_w(void* smem_dst, const CUtensorMap*
       : "memory");
 }
 
+// Eight K=16 steps of one 128-row MMA issued back to back from one elected
+// lane, with every descriptor formed inside the block as base + immediate
+// offset (offsets in 16-byte units, as the descriptor's address fields are).
+//   SS form: A and B are both K-major 128-byte-swizzled tiles of 64-column
+//   boxes; step k advances 32 bytes inside a box and one box every 4 steps.
+__device__ __forceinline__ void mma_ss_k128_w(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                              uint32_t box16) {
+  asm volatile(
+      "{\n\t.reg .pred e, t, f;\n\t.reg .b64 a, b, ab, bb;\n\t"
+      "setp.ne.b32 t, 1, 0;\n\tsetp.ne.b32 f, 0, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, f;\n\t"
+      "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "cvt.u64.u32 ab, %4;\n\t"
+      "add.s64 a, %1, ab;\n\tadd.s64 b, %2, ab;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, a, 2;\n\tadd.s64 b, b, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(box16)
+      : "memory");
+}
+//   TS form (PV): A (P) in TMEM, 8 columns per K=16 step; B (V) MN-major,
+//   16 rows of 128 bytes (128 in 16-byte units) per step.
+__device__ __forceinline__ void mma_ts_k128_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, t, p;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 t, 1, 0;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 a, %1, 8;\n\tadd.s64 b, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+      "add.s32 a, a, 8;\n\tadd.s64 b, b, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
