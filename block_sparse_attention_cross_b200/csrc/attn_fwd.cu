@@ -14,9 +14,9 @@
 //   warp 9      TMEM allocator and MMA issuer
 //   warps 10-11 idle (they complete the control warpgroup)
 // The block is launched with 168 registers per thread.  Inside its own branch
-// the control warpgroup lowers its limit to 88 and the softmax warpgroups
-// raise theirs to 208, which holds a full 128-column score row in registers:
-// 2 * 128 * 208 + 128 * 88 = 384 * 168.
+// the control warpgroup lowers its limit to 56 and the softmax warpgroups
+// raise theirs to 224, which holds a full 128-column score row in registers:
+// 2 * 128 * 224 + 128 * 56 = 384 * 168.
 // The two slots have their own kept-block lists; while one slot's softmax
 // runs, the tensor core works on the other slot's QK^T and PV, so neither
 // waits for the other.  Per slot and block j the MMA issue order is
@@ -42,8 +42,8 @@ namespace {
 constexpr int TILE = 128;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 208;
-constexpr uint32_t kControlRegs = 88;
+constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kControlRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs, "register split");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -408,69 +408,95 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < TILE; ++i)
             if (i >= valid_last) r[i] = f2u(-INFINITY);
         }
-        float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
-#pragma unroll
-        for (int i = 4; i < TILE; i += 8) {
-          mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
-          mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
-          mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
-          mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
-        }
-        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
-        const float m_cand = mx * c2;
-        float alpha = 1.f;
-        if (m_cand > m + kRescaleThreshold) {   // also true for the first block (m = -inf)
-          alpha = ex2_approx(m - m_cand);
-          m = m_cand;
-        }
-        // p = 2^(s c2 - m) two columns at a time (pairs selected by kPolyFrom
+        // p = 2^(s c2 - mref) two columns at a time (pairs selected by kPolyFrom
         // use the FMA-pipe polynomial, the rest the MUFU unit).  P (bf16 pairs)
-        // overwrites the first 64 columns of this slot's S region, 16
-        // columns (32 probabilities) per store.
+        // overwrites the first 64 columns of this slot's S region, 16 columns
+        // (32 probabilities) per store.  Returns the row sum; with `track` it
+        // also returns the row maximum of the raw scores.
         const uint64_t c2x2 = f2pack(c2, c2);
-        const uint64_t negm = f2pack(-m, -m);
-        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+        auto emit_p = [&](float mref, bool track, float& mx_out) -> float {
+          const uint64_t negm = f2pack(-mref, -mref);
+          uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+          float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-        for (int c16 = 0; c16 < TILE / 32; ++c16) {
-          uint32_t pk[16];
+          for (int c16 = 0; c16 < TILE / 32; ++c16) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c16 * 32 + 2 * i;
-            const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
-            uint64_t pv;
-            if ((i & 7) >= kPolyFrom) {
-              pv = exp2_poly2(x);
-            } else {
-              float xl, xh;
-              f2unpack(x, xl, xh);
-              pv = f2pack(ex2_approx(xl), ex2_approx(xh));
+            for (int i = 0; i < 16; ++i) {
+              const int e = c16 * 32 + 2 * i;
+              if (track) {
+                if (i & 1) mxb = fmax3(mxb, u2f(r[e]), u2f(r[e + 1]));
+                else mxa = fmax3(mxa, u2f(r[e]), u2f(r[e + 1]));
+              }
+              const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
+              uint64_t pv;
+              if ((i & 7) >= kPolyFrom) {
+                pv = exp2_poly2(x);
+              } else {
+                float xl, xh;
+                f2unpack(x, xl, xh);
+                pv = f2pack(ex2_approx(xl), ex2_approx(xh));
+              }
+              if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
+              float pl, ph;
+              f2unpack(pv, pl, ph);
+              pk[i] = pack_bf16x2(pl, ph);
             }
-            if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
-            float pl, ph;
-            f2unpack(pv, pl, ph);
-            pk[i] = pack_bf16x2(pl, ph);
+            tmem_st16(t_lane + c16 * 16, pk);
           }
-          tmem_st16(t_lane + c16 * 16, pk);
+          mx_out = fmaxf(mxa, mxb);
+          float a0, a1, b0, b1;
+          f2unpack(acc0, a0, a1);
+          f2unpack(acc1, b0, b1);
+          return (a0 + a1) + (b0 + b1);
+        };
+        float alpha = 1.f;
+        float rs;
+        if (j == 0) {
+          // First block of the tile: the exact row maximum sets the reference.
+          float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
+#pragma unroll
+          for (int i = 4; i < TILE; i += 8) {
+            mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
+            mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
+            mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
+            mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
+          }
+          m = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
+          float unused;
+          rs = emit_p(m, false, unused);
+        } else {
+          // Later blocks: exponentiate against the current reference while
+          // finding the block maximum.  Only if some row's maximum exceeds the
+          // reference by more than the threshold (rare) is the block redone
+          // with the raised reference and O rescaled.
+          float mx;
+          rs = emit_p(m, true, mx);
+          const float m_cand = mx * c2;
+          const bool raise = m_cand > m + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, raise)) {
+            if (raise) {
+              alpha = ex2_approx(m - m_cand);
+              m = m_cand;
+            }
+            tmem_st_wait();   // the speculative P stores land before they are overwritten
+            float unused;
+            rs = emit_p(m, false, unused);
+            // O holds PV(0..j-1) complete: the commit that signalled S(j)
+            // covers every MMA issued before it.
+#pragma unroll
+            for (int q4 = 0; q4 < D / 32; ++q4) {
+              uint32_t ro[32];
+              tmem_ld32(t_lane + 128 + q4 * 32, ro);
+              tmem_ld_wait();
+              reg_fence(ro);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ro[i] = f2u(u2f(ro[i]) * alpha);
+              tmem_st32(t_lane + 128 + q4 * 32, ro);
+            }
+          }
         }
-        float a0, a1, b0, b1;
-        f2unpack(acc0, a0, a1);
-        f2unpack(acc1, b0, b1);
-        const float rs = (a0 + a1) + (b0 + b1);
         l = l * alpha + rs;
-        // O holds PV(0..j-1) complete: the commit that signalled S(j) covers
-        // every MMA issued before it.
-        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
-#pragma unroll
-          for (int q4 = 0; q4 < D / 32; ++q4) {
-            uint32_t r[32];
-            tmem_ld32(t_lane + 128 + q4 * 32, r);
-            tmem_ld_wait();
-            reg_fence(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = f2u(u2f(r[i]) * alpha);
-            tmem_st32(t_lane + 128 + q4 * 32, r);
-          }
-        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&c->p_full[s]);
