@@ -54,6 +54,10 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="skip the density sweep, e2e and CPU baseline")
     p.add_argument("--heads", type=int, default=None,
                    help="use only the first H heads (a smaller case for profiling; default: all 40)")
+    p.add_argument("--workload", default=WORKLOAD, choices=["wan480_25", "wan720_20", "mochi_20", "sweep"],
+                   help="wan480_25 (default, Wan 2.1 480p call, 25%% kept); wan720_20 / mochi_20 (20%% kept); "
+                        "sweep (40 layers x 3 timesteps x 40 heads of the 480p shape, one step = 120 calls, "
+                        "per-map density 0.1-0.6)")
     return p.parse_args()
 
 
@@ -74,6 +78,21 @@ def physical_gpu_id(local):
         if local < len(ids):
             return ids[local]
     return str(local)
+
+
+def max_over_ranks(x, dist, device):
+    """Largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(world, flops_per_rank_step, steps, t_max_ms):
+    """Whole-job TFLOP/s: every rank ran `steps` steps of the same work; the slowest rank sets the time."""
+    return world * flops_per_rank_step * steps / (t_max_ms / 1e3) / 1e12
 
 
 def kept_flops(nnz_blocks, d, B, block=128):
@@ -168,25 +187,31 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-def workload(heads=None):
+SWEEP_LAYERS, SWEEP_STEPS = 40, 3
+
+
+def workload(heads=None, name=WORKLOAD):
     import dataclasses
     from block_sparse_attention_cross_b200 import synthetic as syn
-    w = syn.WORKLOADS[WORKLOAD]
+    w = syn.WORKLOADS["wan480_25" if name == "sweep" else name]
     return dataclasses.replace(w, H=heads) if heads else w
 
 
-def build_workload(device, heads=None, density=None):
+def build_workload(device, heads=None, density=None, name=WORKLOAD):
     import torch
     import block_sparse_attention_cross_b200 as cba
     from block_sparse_attention_cross_b200 import synthetic as syn
-    w = workload(heads)
+    w = workload(heads, name)
     q, k, v = syn.video_qkv(w)
     tensors = []
     for x in (q, k, v):
         bits = syn.f32_to_bf16_bits(x)
         tensors.append(torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16))
     del q, k, v
-    mask = torch.from_numpy(syn.workload_mask(w, density=density)).to(device)
+    if name == "sweep":
+        mask = torch.from_numpy(syn.sweep_masks(w, SWEEP_LAYERS, SWEEP_STEPS)).to(device)
+    else:
+        mask = torch.from_numpy(syn.workload_mask(w, density=density)).to(device)
     bl = cba.compile(mask)
     return w, tensors, bl
 
@@ -201,11 +226,12 @@ def sampled_blocks(w, n_heads, per_head, seed=123):
     return picks
 
 
-def run_oracle_sample(w, qkv_np, mask, picks, scale):
-    """Times the float64 oracle on (head, query block) picks; returns (seconds, kept blocks)."""
+def run_oracle_sample(w, qkv_np, mask, picks, scale, keep_outputs=False):
+    """Times the float64 oracle on (head, query block) picks; returns (seconds, kept blocks, outputs)."""
     import oracle
     q, k, v = qkv_np
     kept = 0
+    outs = []
     t0 = time.perf_counter()
     cache = {}
     for h, qb in picks:
@@ -213,9 +239,11 @@ def run_oracle_sample(w, qkv_np, mask, picks, scale):
             cache.clear()
             cache[h] = tuple(x[:, h:h + 1].astype(np.float64) for x in (q, k, v))
         qh, kh, vh = cache[h]
-        oracle.masked_attention_rows(qh, kh, vh, mask[h:h + 1], w.N, w.block, w.block, scale, 0, 0, qb)
+        o, _ = oracle.masked_attention_rows(qh, kh, vh, mask[h:h + 1], w.N, w.block, w.block, scale, 0, 0, qb)
+        if keep_outputs:
+            outs.append(o)
         kept += int(mask[h, qb].sum())
-    return time.perf_counter() - t0, kept
+    return time.perf_counter() - t0, kept, outs
 
 
 def oracle_inputs(w):
@@ -226,24 +254,49 @@ def oracle_inputs(w):
     return out, mask
 
 
-def cpu_baseline(w, target_seconds=15.0):
-    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1)."""
+def cpu_baseline(w, gpu_out=None, target_seconds=15.0):
+    """The oracle, as it stands, on a bounded sample of the workload (rank 0, N = 1).
+
+    With ``gpu_out`` (the GPU's O for the same inputs) the sampled blocks are
+    also compared element by element and the errors reported.
+    """
     import block_sparse_attention_cross_b200 as cba
     qkv, mask = oracle_inputs(w)
     scale = cba.default_scale(w.d)
     probe = sampled_blocks(w, 1, 4, seed=7)
-    t, kept = run_oracle_sample(w, qkv, mask, probe, scale)
+    t, kept, _ = run_oracle_sample(w, qkv, mask, probe, scale)
     per_block = t / max(1, len(probe))
     per_head = max(2, min(w.nqb, int(target_seconds / max(per_block, 1e-6) / 8)))
     picks = sampled_blocks(w, 8, per_head)
-    t, kept = run_oracle_sample(w, qkv, mask, picks, scale)
-    return {"value": kept_flops(kept, w.d, 1) / t / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{len(picks)} (head, query-block) pairs of the {WORKLOAD} call ({kept} kept blocks, "
-                      f"incl. first and last query block), float64 numpy on {cpu_model()}; {t:.1f} s",
-            "seconds": t}
+    t, kept, outs = run_oracle_sample(w, qkv, mask, picks, scale, keep_outputs=gpu_out is not None)
+    res = {"value": kept_flops(kept, w.d, 1) / t / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+           "sample": f"{len(picks)} (head, query-block) pairs of the {w.name} call ({kept} kept blocks, "
+                     f"incl. first and last query block), float64 numpy on {cpu_model()}; {t:.1f} s",
+           "seconds": t}
+    if gpu_out is not None:
+        errs = []
+        for (h, qb), o in zip(picks, outs):
+            got = gpu_out[0, h, qb * w.block:(qb + 1) * w.block].float().cpu().numpy().astype(np.float64)
+            errs.append(np.abs(got - o).ravel())
+        e = np.concatenate(errs)
+        res["parity_sampled"] = {"max_abs": float(e.max()), "mean_abs": float(e.mean()),
+                                 "bound": {"max_abs": 2e-2, "mean_abs": 2e-3}}
+    return res
 
 
 # ----------------------------------------------------------------------------- GPU arm
+
+def workload_label(name, w, bl):
+    g = w.grid
+    shape = f"{g.frames}x{g.rows}x{g.cols}" + (f" + {g.text_tokens} text" if g.text_tokens else "")
+    if name == "sweep":
+        return (f"sweep: {SWEEP_LAYERS} layers x {SWEEP_STEPS} timesteps x {w.H} heads of the Wan-2.1-14B 480p "
+                f"shape ({shape} = {w.N} tokens, padded {w.Np}, d={w.d}, bf16, 128x128 blocks), one step = "
+                f"{SWEEP_LAYERS * SWEEP_STEPS} calls, per-map density U(0.1, 0.6), mean {100 * bl.density:.1f}% kept")
+    model = {"wan480_25": "Wan-2.1-14B 480p", "wan720_20": "Wan-2.1-14B 720p", "mochi_20": "Mochi-1"}[name]
+    return (f"{name}: {model}-shaped attention call, {shape} = {w.N} tokens (padded {w.Np}), {w.H} heads, "
+            f"d={w.d}, bf16, 128x128 blocks, {100 * bl.density:.1f}% of blocks kept (structured mask)")
+
 
 def time_calls(fn, steps, warmup, torch, dist=None):
     for _ in range(warmup):
@@ -288,13 +341,16 @@ def main_calibatt(args):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    w, (q, k, v), bl = build_workload(dev, args.heads)
+    w, (q, k, v), bl = build_workload(dev, args.heads, name=args.workload)
     out = torch.empty_like(q)
     pk = peaks()
     flops_step = kept_flops(bl.nnz, w.d, w.B)
+    sweep = args.workload == "sweep"
+    offsets = [(l * SWEEP_STEPS + t) * w.H for l in range(SWEEP_LAYERS) for t in range(SWEEP_STEPS)] if sweep else [0]
 
     def step():
-        cba.sparse_attn_fwd(q, k, v, bl, w.N, out=out)
+        for mo in offsets:
+            cba.sparse_attn_fwd(q, k, v, bl, w.N, map_offset=mo, out=out)
 
     warm = max(3, args.warmup)
     launches0 = cba.launch_count()
@@ -306,17 +362,27 @@ def main_calibatt(args):
     total_ms, per = time_calls(step, args.steps, 0, torch, dist)
     clk = clocks.stop()
     launches = cba.launch_count() - launches_warm
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    t_max = float(t.item())
-    value = world * flops_step * args.steps / (t_max / 1e3) / 1e12
+    t_max = max_over_ranks(total_ms, dist, dev)
+    value = weak_scaling_tflops(world, flops_step, args.steps, t_max)
     ms_step = t_max / args.steps
-    per_launch_ms = statistics.mean(per)
-    achieved = flops_step / (per_launch_ms / 1e3) / 1e12
+    per_launch_ms = statistics.mean(per) / len(offsets)
+    achieved = flops_step / len(offsets) / (per_launch_ms / 1e3) / 1e12
 
     extras = {}
-    if not args.no_extras:
+    if sweep:
+        # per-call time against density: one call per (layer, timestep)
+        per, dens_call = [], []
+        for mo in offsets:
+            tc, _ = time_calls(lambda: cba.sparse_attn_fwd(q, k, v, bl, w.N, map_offset=mo, out=out), 3, 1, torch)
+            per.append(tc / 3)
+            dens_call.append(bl.kept_blocks(mo, w.H) / float(w.H * w.nqb * w.nqb))
+        x, y = np.asarray(dens_call), np.asarray(per)
+        slope, icpt = np.polyfit(x, y, 1)
+        r2 = 1.0 - np.sum((y - (slope * x + icpt)) ** 2) / np.sum((y - y.mean()) ** 2)
+        extras["per_call_fit"] = {"ms_per_unit_density": round(float(slope), 4), "intercept_ms": round(float(icpt), 4),
+                                  "r2": round(float(r2), 5), "calls": len(offsets),
+                                  "density_range": [round(float(x.min()), 4), round(float(x.max()), 4)]}
+    if not args.no_extras and not sweep:
         # full-mask run of the same kernel (same inputs) and a density sweep
         full = cba.compile(torch.ones((w.H, w.nqb, w.nqb), dtype=torch.uint8, device=dev))
         tf, _ = time_calls(lambda: cba.sparse_attn_fwd(q, k, v, full, w.N, out=out), 20, 3, torch)
@@ -345,25 +411,22 @@ def main_calibatt(args):
             ho.copy_(out, non_blocking=True)
 
         te, _ = time_calls(e2e_step, 10, 3, torch, dist)
-        te_t = torch.tensor([te], device=dev, dtype=torch.float64)
-        if dist is not None:
-            dist.all_reduce(te_t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te_t.item()) / 10
-        extras["e2e"] = {"value": world * flops_step / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(te, dist, dev) / 10
+        extras["e2e"] = {"value": weak_scaling_tflops(world, flops_step, 1, e2e_ms), "unit": UNIT,
                          "h2d_bytes_per_step": int(3 * q.numel() * q.element_size()),
                          "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms}
 
+    if rank == 0 and sweep:
+        extras["calls_per_step"] = len(offsets)
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": warm, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD}: Wan-2.1-14B-shaped attention call, 21x30x52 = 32760 tokens "
-                                   f"(padded {w.Np}), {w.H} heads, d={w.d}, bf16, 128x128 blocks, "
-                                   f"{100 * bl.density:.1f}% of blocks kept (structured mask)",
+            "config": {"workload": workload_label(args.workload, w, bl),
                        "B": w.B, "H": w.H, "N": w.N, "Np": w.Np, "d": w.d, "block": w.block,
                        "kept_blocks": bl.nnz, "density": round(bl.density, 6),
-                       "l2": "inputs 1.0 GB > 126 MB L2; no flush between steps",
+                       "l2": f"inputs {3 * q.numel() * 2 / 1e9:.2f} GB > 126 MB L2; no flush between steps",
                        "parallelism": f"replicas x{world} (head-sharded work is independent)"},
             "pct_bf16_peak_burst": round(100 * value / world / pk["bf16_burst"], 2),
             "pct_bf16_peak_sustained": round(100 * value / world / pk["bf16_sustained"], 2),
@@ -373,15 +436,17 @@ def main_calibatt(args):
                          "traffic": kernel_traffic(),
                          "kernel": "k_attn_fwd<128>",
                          "peak_kind": f"bf16_tflops_sustained ({pk['source']}); burst {pk['bf16_burst']}",
-                         "algorithmic_flops_per_launch": flops_step},
+                         "algorithmic_flops_per_launch": flops_step / len(offsets)},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
         line.update({k2: v2 for k2, v2 in extras.items() if k2 != "e2e"})
         if "e2e" in extras:
             line["e2e"] = extras["e2e"]
-        if world == 1 and not args.no_extras:
-            line["cpu_baseline"] = cpu_baseline(w)
+        if world == 1 and not args.no_extras and not sweep:
+            cba.sparse_attn_fwd(q, k, v, bl, w.N, out=out)
+            torch.cuda.synchronize()
+            line["cpu_baseline"] = cpu_baseline(w, out)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -395,12 +460,12 @@ def main_reference(args):
     if rank != 0:
         return
     import block_sparse_attention_cross_b200 as cba  # noqa: F401  (scale helper only)
-    w = workload(args.heads)
+    w = workload(args.heads, "wan480_25" if args.workload == "sweep" else args.workload)
     qkv, mask = oracle_inputs(w)
     scale = cba.default_scale(w.d)
     steps, warm = args.steps, max(3, args.warmup)
     probe = sampled_blocks(w, 1, 2, seed=3)
-    t_probe, _ = run_oracle_sample(w, qkv, mask, probe, scale)
+    t_probe, _, _ = run_oracle_sample(w, qkv, mask, probe, scale)
     per_block = t_probe / len(probe)
     budget = 150.0  # seconds for warmup + timed steps
     blocks_per_step = max(1, int(budget / (steps + warm) / max(per_block, 1e-6)))
@@ -408,7 +473,8 @@ def main_reference(args):
 
     def one_step():
         picks = [(int(rng.integers(w.H)), int(rng.integers(w.nqb))) for _ in range(blocks_per_step)]
-        return run_oracle_sample(w, qkv, mask, picks, scale)
+        t, kept, _ = run_oracle_sample(w, qkv, mask, picks, scale)
+        return t, kept
 
     for _ in range(warm):
         one_step()
@@ -422,7 +488,7 @@ def main_reference(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": warm,
         "ms_per_step": 1e3 * tot_t / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": f"{WORKLOAD} (sampled query blocks per step)", "B": w.B, "H": w.H, "N": w.N,
+        "config": {"workload": f"{w.name} (sampled query blocks per step)", "B": w.B, "H": w.H, "N": w.N,
                    "Np": w.Np, "d": w.d, "block": w.block, "density": w.density,
                    "blocks_per_step": blocks_per_step},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",

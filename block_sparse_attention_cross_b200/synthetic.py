@@ -311,3 +311,20 @@ def workload_mask(w: Workload, density=None, n_maps=None, seed=None):
         period = 13
     return structured_block_mask(n_maps, w.nqb, nkb, dens, seed, g.cols, g.rows * g.cols,
                                  block=w.block, period=period, forced_cols=forced)
+
+
+def sweep_masks(w: Workload, layers=40, timesteps=3, seed=1000, lo=0.1, hi=0.6):
+    """Mask dictionary of a denoising-step sweep: one structured mask per (layer, timestep, head).
+
+    Map id = (layer * timesteps + t) * H + head; map m has density ~ U(lo, hi)
+    (one draw per map from ``seed``) and its own structure seed ``seed + m``.
+    """
+    n_maps = layers * timesteps * w.H
+    dens = np.random.default_rng(seed).uniform(lo, hi, n_maps)
+    g = w.grid
+    out = np.empty((n_maps, w.nqb, w.nqb), dtype=np.uint8)
+    for m in range(n_maps):
+        out[m] = structured_block_mask(1, w.nqb, w.nqb, dens[m], seed + m, g.cols, g.rows * g.cols,
+                                       block=w.block)[0]
+    return out
+

@@ -169,3 +169,36 @@ def test_bf16_persistent_schedule_ragged_lists(d):
             if cnt:
                 mask[h, qb, rng.choice(nb, size=cnt, replace=False)] = 1
     run_full_compare(q, k, v, mask, N, 128, "bf16", d)
+
+
+@pytest.mark.slow
+def test_bf16_sweep_dictionary_calls_sampled():
+    # 40 layers x 3 timesteps x 40 heads of the Wan 480p shape, each map with
+    # its own density in [0.1, 0.6]; a call uses the 40 maps of one
+    # (layer, timestep) through map_offset.
+    w = syn.WORKLOADS["wan480_25"]
+    masks = syn.sweep_masks(w, 40, 3)
+    q, k, v = syn.video_qkv(w)
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    v64, vd = bf16_pair(v)
+    del q, k, v
+    bl = cba.compile(torch.from_numpy(masks).cuda())
+    assert bl.nnz == int(masks.sum())
+    scale = cba.default_scale(w.d)
+    rng = np.random.default_rng(4)
+    for layer, t in ((0, 0), (17, 2), (39, 1)):
+        mo = (layer * 3 + t) * w.H
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, w.N, scale=scale, map_offset=mo, return_lse=True, status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        errs = []
+        for h, qb in [(0, 0), (w.H - 1, w.nqb - 1)] + [(int(rng.integers(w.H)), int(rng.integers(w.nqb)))
+                                                       for _ in range(6)]:
+            O, L = oracle.masked_attention_rows(q64, k64, v64, masks[mo:mo + w.H], w.N, 128, 128, scale, 0, h, qb)
+            rows = slice(qb * 128, (qb + 1) * 128)
+            errs.append(np.abs(to_np64(o[0, h, rows]) - O).ravel())
+            assert_lse(lse[0, h, rows].cpu().numpy(), L, 1e-3)
+        err = np.concatenate(errs)
+        assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (layer, t, err.max(), err.mean())

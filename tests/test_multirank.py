@@ -1,0 +1,65 @@
+"""Host-side logic of the multi-rank benchmark, run as two gloo ranks on CPU.
+
+Every rank runs its own replica of the workload (the path shards by head and
+has no data exchange); the only collective is the timing reduction, whose
+maximum over ranks sets the whole-job throughput.
+"""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        assert bench.dist_env() == (world, rank, rank)
+        local_ms = [100.0, 125.0][rank]
+        t_max = bench.max_over_ranks(local_ms, dist, torch.device("cpu"))
+        value = bench.weak_scaling_tflops(world, 5.0e12, 10, t_max)
+        out[rank] = (t_max, value)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_gloo():
+    world = 2
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    for rank in range(world):
+        t_max, value = out[rank]
+        assert t_max == 125.0
+        assert value == pytest.approx(2 * 5.0e12 * 10 / 0.125 / 1e12)
+
+
+def test_single_rank_helpers_without_process_group():
+    assert bench.max_over_ranks(3.5, None, None) == 3.5
+    assert bench.weak_scaling_tflops(1, 1e12, 1, 1000.0) == pytest.approx(1.0)
+
+
+def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setattr(bench, "oracle_inputs", lambda w: (_ for _ in ()).throw(AssertionError("rank 1 worked")))
+
+    class A:
+        steps, warmup, heads, workload = 3, 3, None, "wan480_25"
+
+    bench.main_reference(A())
+    assert capsys.readouterr().out == ""
