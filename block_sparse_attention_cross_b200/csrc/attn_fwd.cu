@@ -48,7 +48,10 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchR
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// The reference max is raised (and O rescaled) only when a block's row max
+// exceeds it by more than this many log2 units, so every P <= 2^64; row sums
+// and O stay far below the fp32 range for |v| < 2^47.
+constexpr float kRescaleThreshold = 64.0f;
 // Column pairs i with (i % 8) >= kPolyFrom evaluate exp2 with the FMA-pipe
 // polynomial instead of MUFU.  Measured on B200 at this instruction mix the
 // MUFU unit is not the limiter, so the polynomial is off (8).
@@ -85,6 +88,7 @@ struct TileList {
   int n;      // kept blocks (0 for an empty or rejected list)
   int base;   // first kept block
   int p0;     // start of the pattern in pat_off
+  int rot;    // blocks are walked from list index rot (first kept block >= qb), wrapping around
 };
 
 // Reads and checks the kept-block list of work tile t.  Warp-collective: every
@@ -120,6 +124,15 @@ __device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool repor
   if (bad && report && lane == 0) report_status(a.status, CALIBATT_E_CORRUPT);
   tl.n = bad ? 0 : n;
   tl.p0 = p0;
+  // Walk order: start at the query tile's own (diagonal) block, or the first
+  // kept block after it, and wrap around.  For video attention the query's
+  // own block usually holds the row maximum, so later blocks rarely raise it.
+  int below = 0;
+  for (int i0 = 0; i0 < tl.n; i0 += 32) {
+    const int i = i0 + lane;
+    below += __popc(__ballot_sync(0xffffffffu, i < tl.n && tl.base + a.pat_off[p0 + i] < tl.qb));
+  }
+  tl.rot = (below < tl.n) ? below : 0;
   return tl;
 }
 
@@ -128,7 +141,7 @@ __device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool repor
 // tiles with empty lists.  A step of a slot is "PV of the previous block (if
 // any), then QK^T of the next block (if any)".
 struct SlotSched {
-  int t, n, base, p0, bh, j, pv;
+  int t, n, base, p0, bh, j, pv, rot;
   bool done;
 };
 
@@ -140,6 +153,7 @@ __device__ __forceinline__ void sched_next_tile(const TcArgs& a, SlotSched& st, 
       st.base = tl.base;
       st.p0 = tl.p0;
       st.bh = tl.bh;
+      st.rot = tl.rot;
       st.j = 0;
       st.pv = -1;
       return;
@@ -215,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         SlotSched& q = st[s];
         if (q.done) continue;
         if (q.pv >= 0) {
-          const int kb = q.base + a.pat_off[q.p0 + q.pv];
+          const int kb = q.base + a.pat_off[q.p0 + (q.pv + q.rot) % q.n];
           const int row = q.bh * a.Np + kb * TILE;
           const int e = g % R;
           ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
@@ -249,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           ++qfills[s];
         }
-        const int kb = q.base + a.pat_off[q.p0 + j];
+        const int kb = q.base + a.pat_off[q.p0 + (j + q.rot) % q.n];
         const int row = q.bh * a.Np + kb * TILE;
         const int e = g % R;
         ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
@@ -388,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
       const int valid_last = (kb_last == a.nkb - 1) ? (a.N - kb_last * TILE) : TILE;
+      const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
       float m = -INFINITY;
       float l = 0.f;
       for (int j = 0; j < tl.n; ++j) {
@@ -402,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(t_lane + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
         tmem_ld_wait();
         reg_fence(r);
-        if (j == tl.n - 1 && valid_last < TILE) {
+        if (j == j_last && valid_last < TILE) {
           // Key columns past the sequence end exist only in the last block.
 #pragma unroll
           for (int i = 0; i < TILE; ++i)
