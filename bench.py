@@ -390,15 +390,15 @@ def main_calibatt(args):
         extras["speedup_vs_full_mask"] = t_full / ms_step
         extras["full_mask_ms"] = t_full
         extras["full_mask_tflops"] = kept_flops(full.nnz, w.d, w.B) / (t_full / 1e3) / 1e12
-        sweep = []
+        dens_sweep = []
         for dens in (1.0, 0.8, 0.6, 0.4, 0.25, 0.2, 0.1):
             from block_sparse_attention_cross_b200 import synthetic as syn
             m = torch.from_numpy(syn.workload_mask(w, density=dens)).to(dev) if dens < 1.0 else None
             b = cba.compile(m) if m is not None else full
             td, _ = time_calls(lambda: cba.sparse_attn_fwd(q, k, v, b, w.N, out=out), 20, 3, torch)
-            sweep.append({"density": round(b.density, 4), "ms": round(td / 20, 4),
+            dens_sweep.append({"density": round(b.density, 4), "ms": round(td / 20, 4),
                           "kept_tflops": round(kept_flops(b.nnz, w.d, w.B) / (td / 20 / 1e3) / 1e12, 1)})
-        extras["density_sweep"] = sweep
+        extras["density_sweep"] = dens_sweep
         # end to end through the public API with host buffers
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         ho = torch.empty_like(hq).pin_memory()
