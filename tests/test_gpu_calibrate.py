@@ -43,6 +43,7 @@ def test_block_energy(dtype, d, block):
     Eo = oracle.block_energy(q64, k64, w.N, block, block, scale)
     nreal = -(-w.N // block)
     rel = np.abs(E - Eo).max()
+    print(f"PARITY energy {dtype} d={d} block={block} max_abs={rel:.3e}")
     assert rel <= (1e-5 if dtype == "fp32" else 5e-5), rel
     np.testing.assert_allclose(E[:, :nreal].sum(axis=-1), 1.0, atol=1e-4)
 
@@ -103,6 +104,7 @@ def test_calibrate_small_end_to_end():
     for E in Eo:
         tie |= near_tie_rows(E, k)
     diff_rows = (mask.cpu().numpy() != m64).any(axis=-1)
+    print(f"PARITY calibrate rows_differing={int(diff_rows.sum())} near_tie_rows={int(tie.sum())} of {tie.size}")
     assert not (diff_rows & ~tie).any()
     # the compiled calibrated mask drives the forward kernel
     bl = cba.compile(mask)
@@ -128,3 +130,4 @@ def test_calibrate_wan_config_subset():
     assert np.array_equal(votes.cpu().numpy(), v_o)
     assert np.array_equal(mask.cpu().numpy(), m_o)
     np.testing.assert_allclose(np.stack(Eg)[:, :, :, :].sum(axis=-1), 1.0, atol=2e-3)
+    print(f"PARITY calibrate-wan480 8 inputs: votes and masks bit-exact; mask density {float(mask.float().mean()):.4f}")

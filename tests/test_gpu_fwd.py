@@ -41,6 +41,7 @@ def run_full_compare(q, k, v, mask, N, block, dtype, d, B=1, H=None, map_offset=
     else:
         mx, mn = assert_close(to_np64(o), O, FP32_MAX_ABS)
         assert_lse(lse.cpu().numpy(), L, lse_tol or 1e-5)
+    print(f"PARITY {dtype} N={N} d={d} block={block} max_abs={mx:.3e} mean_abs={mn:.3e}")
     return mx, mn
 
 
@@ -133,6 +134,7 @@ def sampled_parity(w, mask, qkv=None, n_samples=24, seed=0, map_offset=0):
         assert_lse(lse[0, h, rows].cpu().numpy(), L, 1e-3)
     err = np.concatenate([e.ravel() for e in errs])
     assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
+    print(f"PARITY {w.name} sampled {len(picks)} query blocks max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
     return err.max(), err.mean()
 
 
@@ -202,3 +204,4 @@ def test_bf16_sweep_dictionary_calls_sampled():
             assert_lse(lse[0, h, rows].cpu().numpy(), L, 1e-3)
         err = np.concatenate(errs)
         assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (layer, t, err.max(), err.mean())
+        print(f"PARITY sweep layer={layer} t={t} max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
