@@ -153,6 +153,49 @@ def sparse_attn_fwd(q, k, v, bl: BlockList, N, scale=None, map_offset=0, return_
     return (out, lse) if return_lse else out
 
 
+def _need_host(*ts):
+    for t in ts:
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("host tensors must be contiguous CPU tensors (pin_memory() for overlap)")
+
+
+def sparse_attn_fwd_streamed(q, k, v, bl: BlockList, N, staging, scale=None, map_offset=0, heads_per_chunk=8,
+                             out=None, lse=None, status=None):
+    """Block-sparse attention forward for q, k, v in host memory.
+
+    q, k, v: [B, H, Np, d] bf16 or fp32 CPU tensors (pinned for overlap).
+    ``staging``: (q_dev, k_dev, v_dev, o_dev[, lse_dev]) CUDA tensors of the
+    same shapes, owned by the caller and overwritten.  Heads are processed in
+    chunks of ``heads_per_chunk``; each chunk's host -> device copies, kernel
+    and device -> host copy overlap those of the neighbouring chunks.  The
+    result lands in ``out`` (a host tensor, allocated pinned when not given)
+    and ``lse`` (host float32 [B, H, Np], only if given) once the current CUDA
+    stream has been synchronised.  Returns ``out``.
+    """
+    _need_host(q, k, v, out, lse)
+    B, H, Np, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    qd, kd, vd, od = staging[:4]
+    lse_d = staging[4] if len(staging) > 4 else None
+    if (lse is None) != (lse_d is None):
+        raise ValueError("pass lse together with an lse staging buffer")
+    _need_cuda(qd, kd, vd, od, lse_d, status)
+    for t in (qd, kd, vd, od):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("staging buffers must match q's shape and dtype")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    s = bl.as_struct()
+    with torch.cuda.device(qd.device):
+        check(load().calibatt_sparse_attn_fwd_streamed(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(qd), _ptr(kd), _ptr(vd), _ptr(od), _ptr(lse_d),
+            B, H, int(N), Np, d, _dtype_code(q), scale, ctypes.byref(s), int(map_offset), int(heads_per_chunk),
+            _ptr(status), _stream(qd.device)))
+    return out
+
+
 def _calib_workspace(H, N, Np, d, bq, bk, device):
     n = ctypes.c_size_t(0)
     check(load().calibatt_calibrate_workspace_size(H, int(N), Np, d, bq, bk, ctypes.byref(n)))

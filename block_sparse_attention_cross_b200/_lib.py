@@ -39,6 +39,10 @@ EXPORTS = {
     "calibatt_get_spin_limit_ns": (c_uint64, []),
     "calibatt_sparse_attn_fwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                          c_int, c_int, c_int, c_float, c_void_p, c_int, c_void_p, c_void_p]),
+    "calibatt_sparse_attn_fwd_streamed": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                  c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                                  c_int, c_int, c_int, c_float, c_void_p, c_int, c_int, c_void_p,
+                                                  c_void_p]),
     "calibatt_block_energy": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "calibatt_block_energy_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,

@@ -134,24 +134,12 @@ int validate_blocklist(const calibatt_blocklist* bl) {
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-const char* calibatt_last_error(void) { return g_last_error.c_str(); }
-
-int calibatt_version(void) { return 1 * 10000 + 0 * 100 + 0; }
-
-uint64_t calibatt_launch_count(void) { return g_launches.load(); }
-
-void calibatt_set_spin_limit_ns(uint64_t ns) {
-  spin_limit_ns();
-  g_spin_ns.store(ns > 0 ? ns : 1);
-}
-
-uint64_t calibatt_get_spin_limit_ns(void) { return spin_limit_ns(); }
-
-int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-                             int Np, int d, int dtype, float scale, const calibatt_blocklist* bl, int map_offset,
-                             int32_t* dev_status, calibatt_stream_t stream) {
+// Argument checks of the forward, shared by the plain and the streamed entry
+// points so that neither enqueues anything for a call it would reject.
+int check_fwd(const void* q, const void* k, const void* v, const void* o, int B, int H, int N, int Np, int d,
+              int dtype, float scale, const calibatt_blocklist* bl, int map_offset) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
     return set_error(CALIBATT_E_INVALID, "q, k, v and o must be non-NULL");
   if (B <= 0 || H <= 0 || N <= 0 || Np < N || d <= 0)
@@ -172,12 +160,86 @@ int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
     return set_error(CALIBATT_E_INVALID, "map_offset %d + H %d exceeds n_maps %d", map_offset, H, bl->n_maps);
   if (static_cast<long long>(B) * H * Np >= (1ll << 31))
     return set_error(CALIBATT_E_UNSUPPORTED, "B*H*Np must be below 2^31 rows");
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
   if (dtype == CALIBATT_BF16) {
     if (!(d == 64 || d == 128) || bl->block_q != 128 || bl->block_k != 128)
       return set_error(CALIBATT_E_UNSUPPORTED, "bf16 path supports d in {64,128} with 128x128 blocks");
     if (nkb > 1024) return set_error(CALIBATT_E_UNSUPPORTED, "at most 1024 key blocks per row");
+    return CALIBATT_OK;
+  }
+  if (dtype == CALIBATT_FP32) {
+    if (!(d == 64 || d == 128) || !(bl->block_q == 64 || bl->block_q == 128) ||
+        !(bl->block_k == 64 || bl->block_k == 128))
+      return set_error(CALIBATT_E_UNSUPPORTED, "fp32 path supports d in {64,128}, blocks in {64,128}");
+    if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
+    return CALIBATT_OK;
+  }
+  return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
+}
+
+}  // namespace
+
+namespace {
+
+// Copy streams and events of the streamed forward, one set per device,
+// created on first use and kept for the life of the process.  The mutex makes
+// each call's record/wait sequence atomic, so concurrent callers never see
+// each other's event records.
+struct StreamSet {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
+};
+std::mutex g_stream_mu;
+StreamSet g_streams[64];
+
+int stream_set(StreamSet** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("cudaGetDevice");
+  StreamSet& ss = g_streams[dev];
+  if (ss.h2d == nullptr) {
+    if (cudaStreamCreateWithFlags(&ss.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&ss.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.start, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.in, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.out, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.done, cudaEventDisableTiming) != cudaSuccess) {
+      ss = StreamSet{};
+      return check_launch("creating the copy streams");
+    }
+  }
+  *out = &ss;
+  return CALIBATT_OK;
+}
+
+int cuda_ok(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return CALIBATT_OK;
+  return set_error(CALIBATT_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* calibatt_last_error(void) { return g_last_error.c_str(); }
+
+int calibatt_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+uint64_t calibatt_launch_count(void) { return g_launches.load(); }
+
+void calibatt_set_spin_limit_ns(uint64_t ns) {
+  spin_limit_ns();
+  g_spin_ns.store(ns > 0 ? ns : 1);
+}
+
+uint64_t calibatt_get_spin_limit_ns(void) { return spin_limit_ns(); }
+
+int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                             int Np, int d, int dtype, float scale, const calibatt_blocklist* bl, int map_offset,
+                             int32_t* dev_status, calibatt_stream_t stream) {
+  int rc = check_fwd(q, k, v, o, B, H, N, Np, d, dtype, scale, bl, map_offset);
+  if (rc) return rc;
+  const int nqb = Np / bl->block_q, nkb = Np / bl->block_k;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == CALIBATT_BF16) {
     TcArgs a{};
     a.B = B; a.H = H; a.N = N; a.Np = Np; a.nqb = nqb; a.nkb = nkb;
     a.scale_log2 = scale * 1.4426950408889634f;
@@ -186,20 +248,79 @@ int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
     a.o = o; a.lse = lse; a.status = dev_status; a.spin_ns = spin_limit_ns();
     return launch_tc_fwd(q, k, v, d, a, s);
   }
-  if (dtype == CALIBATT_FP32) {
-    if (!(d == 64 || d == 128) || !(bl->block_q == 64 || bl->block_q == 128) ||
-        !(bl->block_k == 64 || bl->block_k == 128))
-      return set_error(CALIBATT_E_UNSUPPORTED, "fp32 path supports d in {64,128}, blocks in {64,128}");
-    if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
-    SimtArgs a{};
-    a.B = B; a.H = H; a.N = N; a.Np = Np; a.block_q = bl->block_q; a.block_k = bl->block_k;
-    a.nqb = nqb; a.nkb = nkb; a.scale = scale;
-    a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
-    a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
-    a.lse = lse; a.status = dev_status;
-    return launch_simt_fwd(q, k, v, o, d, a, s);
+  SimtArgs a{};
+  a.B = B; a.H = H; a.N = N; a.Np = Np; a.block_q = bl->block_q; a.block_k = bl->block_k;
+  a.nqb = nqb; a.nkb = nkb; a.scale = scale;
+  a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
+  a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
+  a.lse = lse; a.status = dev_status;
+  return launch_simt_fwd(q, k, v, o, d, a, s);
+}
+
+int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                      float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                      float* lse_dev, int B, int H, int N, int Np, int d, int dtype, float scale,
+                                      const calibatt_blocklist* bl, int map_offset, int heads_per_chunk,
+                                      int32_t* dev_status, calibatt_stream_t stream) {
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || o_host == nullptr)
+    return set_error(CALIBATT_E_INVALID, "q_host, k_host, v_host and o_host must be non-NULL");
+  if (q_dev == nullptr || k_dev == nullptr || v_dev == nullptr || o_dev == nullptr)
+    return set_error(CALIBATT_E_INVALID, "q_dev, k_dev, v_dev and o_dev must be non-NULL");
+  if ((lse_host == nullptr) != (lse_dev == nullptr))
+    return set_error(CALIBATT_E_INVALID, "lse_host and lse_dev must both be given or both be NULL");
+  if (heads_per_chunk <= 0) return set_error(CALIBATT_E_INVALID, "heads_per_chunk must be >= 1");
+  int rc = check_fwd(q_dev, k_dev, v_dev, o_dev, B, H, N, Np, d, dtype, scale, bl, map_offset);
+  if (rc) return rc;
+  const size_t esize = dtype == CALIBATT_BF16 ? 2 : 4;
+  const size_t plane = static_cast<size_t>(Np) * d * esize;   // bytes of one (b, h) slice
+  const int hc = heads_per_chunk < H ? heads_per_chunk : H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  std::lock_guard<std::mutex> lock(g_stream_mu);
+  StreamSet* ss = nullptr;
+  rc = stream_set(&ss);
+  if (rc) return rc;
+  // The staging buffers may still be in use by work already on `stream`.
+  if ((rc = cuda_ok(cudaEventRecord(ss->start, s), "cudaEventRecord")) ||
+      (rc = cuda_ok(cudaStreamWaitEvent(ss->h2d, ss->start, 0), "cudaStreamWaitEvent")) ||
+      (rc = cuda_ok(cudaStreamWaitEvent(ss->d2h, ss->start, 0), "cudaStreamWaitEvent")))
+    return rc;
+  for (int b = 0; b < B; ++b) {
+    for (int h0 = 0; h0 < H; h0 += hc) {
+      const int hn = (H - h0) < hc ? (H - h0) : hc;
+      const size_t first = static_cast<size_t>(b) * H + h0;      // first (b, h) slice of the chunk
+      const size_t off = first * plane, bytes = static_cast<size_t>(hn) * plane;
+      const size_t loff = first * Np, lbytes = static_cast<size_t>(hn) * Np * sizeof(float);
+      auto at = [](const void* p, size_t o) { return static_cast<const char*>(p) + o; };
+      auto atw = [](void* p, size_t o) { return static_cast<char*>(p) + o; };
+      if ((rc = cuda_ok(cudaMemcpyAsync(atw(q_dev, off), at(q_host, off), bytes, cudaMemcpyHostToDevice, ss->h2d),
+                        "cudaMemcpyAsync(q)")) ||
+          (rc = cuda_ok(cudaMemcpyAsync(atw(k_dev, off), at(k_host, off), bytes, cudaMemcpyHostToDevice, ss->h2d),
+                        "cudaMemcpyAsync(k)")) ||
+          (rc = cuda_ok(cudaMemcpyAsync(atw(v_dev, off), at(v_host, off), bytes, cudaMemcpyHostToDevice, ss->h2d),
+                        "cudaMemcpyAsync(v)")) ||
+          (rc = cuda_ok(cudaEventRecord(ss->in, ss->h2d), "cudaEventRecord")) ||
+          (rc = cuda_ok(cudaStreamWaitEvent(s, ss->in, 0), "cudaStreamWaitEvent")))
+        return rc;
+      rc = calibatt_sparse_attn_fwd(atw(q_dev, off), atw(k_dev, off), atw(v_dev, off), atw(o_dev, off),
+                                    lse_dev ? lse_dev + loff : nullptr, 1, hn, N, Np, d, dtype, scale, bl,
+                                    map_offset + h0, dev_status, stream);
+      if (rc) return rc;
+      if ((rc = cuda_ok(cudaEventRecord(ss->out, s), "cudaEventRecord")) ||
+          (rc = cuda_ok(cudaStreamWaitEvent(ss->d2h, ss->out, 0), "cudaStreamWaitEvent")) ||
+          (rc = cuda_ok(cudaMemcpyAsync(atw(o_host, off), at(o_dev, off), bytes, cudaMemcpyDeviceToHost, ss->d2h),
+                        "cudaMemcpyAsync(o)")))
+        return rc;
+      if (lse_host != nullptr &&
+          (rc = cuda_ok(cudaMemcpyAsync(lse_host + loff, lse_dev + loff, lbytes, cudaMemcpyDeviceToHost, ss->d2h),
+                        "cudaMemcpyAsync(lse)")))
+        return rc;
+    }
   }
-  return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
+  if ((rc = cuda_ok(cudaEventRecord(ss->done, ss->d2h), "cudaEventRecord")) ||
+      (rc = cuda_ok(cudaStreamWaitEvent(s, ss->done, 0), "cudaStreamWaitEvent")))
+    return rc;
+  return CALIBATT_OK;
 }
 
 int calibatt_calibrate_workspace_size(int H, int N, int Np, int d, int block_q, int block_k, size_t* bytes) {

@@ -54,7 +54,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 64.0f;
 // Column pairs i with (i % 8) >= kPolyFrom evaluate exp2 with the FMA-pipe
 // polynomial instead of MUFU.  Measured on B200 at this instruction mix the
-// MUFU unit is not the limiter, so the polynomial is off (8).
+// MUFU unit is not the limiter, so the polynomial is off (8).  The epilogue's
+// normaliser fix-up re-forms one probability with MUFU, so it is exact only
+// while the polynomial is off.
 constexpr int kPolyFrom = 8;
 
 template <int D>
@@ -405,6 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
       float m = -INFINITY;
       float l = 0.f;
+      // Largest raw score of the row so far (for the normalisation fix-up in
+      // the epilogue).
+      float s_best = -INFINITY;
       for (int j = 0; j < tl.n; ++j) {
         ok = mbar_wait(&c->s_full[s], sc & 1, &c->abort, a.spin_ns);
         ok = __all_sync(0xffffffffu, ok);
@@ -477,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
             mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
           }
-          m = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * c2;
+          s_best = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+          m = s_best * c2;
           float unused;
           rs = emit_p(m, false, unused);
         } else {
@@ -489,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs = emit_p(m, true, mx);
           const float m_cand = mx * c2;
           const bool raise = m_cand > m + kRescaleThreshold;
+          s_best = fmaxf(s_best, mx);
           if (__any_sync(0xffffffffu, raise)) {
             if (raise) {
               alpha = ex2_approx(m - m_cand);
@@ -523,8 +530,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       ++tiles;
       tc_fence_after();
+      // O holds sums of bf16-rounded probabilities while l sums the fp32 ones.
+      // Their mismatch is negligible except for a dominant probability, which
+      // is not exactly representable once the reference lags the row maximum
+      // (threshold above): its rounding error, recomputed here exactly as the
+      // softmax formed it, is moved into the normaliser so that a row with one
+      // dominant key returns that key's value.  The row's largest score was
+      // always exponentiated against the final reference m: a raise after its
+      // block would need a larger score, and a raise in its block redoes the
+      // block against that very score (p = 1, exact).  The LSE keeps the fp32
+      // sum.
+      const float p_best = ex2_approx(fmaf(s_best, c2, -m));
+      const float l_o = l + (__uint_as_float(pack_bf16x2(p_best, 0.f) << 16) - p_best);
       const bool pad_row = grow >= a.N;
-      const float inv_l = pad_row ? 0.f : 1.f / l;
+      const float inv_l = pad_row ? 0.f : 1.f / l_o;
 #pragma unroll
       for (int q4 = 0; q4 < D / 32; ++q4) {
         uint32_t r[32];

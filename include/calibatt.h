@@ -140,6 +140,42 @@ int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
                              int32_t* dev_status, calibatt_stream_t stream);
 
 /*
+ * calibatt_sparse_attn_fwd_streamed -- the forward above for inputs and
+ * output in host memory.
+ *
+ * Computes exactly what calibatt_sparse_attn_fwd computes (same kernel, same
+ * results bit for bit), one chunk of heads at a time: the chunk's Q, K, V are
+ * copied host -> device on an internal copy stream, the forward of the chunk
+ * runs on `stream`, and its O (and LSE) are copied device -> host on a second
+ * copy stream, so the copies of one chunk overlap the compute of its
+ * neighbours.
+ *  q_host, k_host, v_host  [B, H, Np, d] of `dtype` in host memory (read);
+ *                    page-locked memory is needed for the copies to overlap.
+ *  o_host            [B, H, Np, d] host memory (written); lse_host [B, H, Np]
+ *                    float32 host memory or NULL.
+ *  q_dev, k_dev, v_dev, o_dev  device staging buffers of the same shape,
+ *                    owned by the caller (16-byte aligned; overwritten);
+ *                    lse_dev [B, H, Np] float32 device, non-NULL exactly when
+ *                    lse_host is.
+ *  heads_per_chunk   heads per chunk (>= 1; clamped to H); chunks never span
+ *                    two batch entries.
+ * The other arguments are those of calibatt_sparse_attn_fwd and are checked
+ * before anything is enqueued.  The copy streams are ordered after the work
+ * already on `stream`, and on return `stream` is ordered after every copy of
+ * this call: synchronise `stream` before reading o_host.  The copy streams
+ * and their events are created on first use (per device) and kept; calls
+ * from several host threads are serialised while they enqueue.
+ * Errors: CALIBATT_E_INVALID / E_UNSUPPORTED as calibatt_sparse_attn_fwd
+ * (nothing enqueued); CALIBATT_E_CUDA if a copy or event call fails (work
+ * enqueued before the failure stays enqueued).
+ */
+int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                      float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                      float* lse_dev, int B, int H, int N, int Np, int d, int dtype, float scale,
+                                      const calibatt_blocklist* bl, int map_offset, int heads_per_chunk,
+                                      int32_t* dev_status, calibatt_stream_t stream);
+
+/*
  * calibatt_block_energy -- block energies of one calibration input.
  *
  * Paper page, Figure 2 (block-level post-softmax attention maps) and

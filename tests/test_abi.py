@@ -95,6 +95,31 @@ def test_fwd_rejects_mismatched_blocklist_and_unsupported(lib):
     assert lib.calibatt_sparse_attn_fwd(*args(1, 2, 896, 1024, 128, _lib.BF16, 0)) == _lib.E_INVALID
 
 
+def test_streamed_fwd_checks_everything_before_enqueueing(lib):
+    # Every rejection below happens on the host before any stream, event or
+    # copy is created, so no CUDA call is made.
+    fake = ctypes.c_void_p(0x10000)
+    host = ctypes.c_void_p(0x30000)
+    bl = _blocklist(2, 8, 8, 128, 128)
+
+    def call(qh=host, oh=host, lh=None, qd=fake, ld=None, B=1, H=2, N=1000, Np=1024, d=128, dt=_lib.BF16, mo=0,
+             hpc=1, blp=ctypes.byref(bl)):
+        return lib.calibatt_sparse_attn_fwd_streamed(qh, host, host, oh, lh, qd, fake, fake, fake, ld, B, H, N, Np,
+                                                     d, dt, 0.1, blp, mo, hpc, None, None)
+
+    assert call(qh=None) == _lib.E_INVALID and "host" in _err(lib)
+    assert call(oh=None) == _lib.E_INVALID
+    assert call(qd=None) == _lib.E_INVALID and "dev" in _err(lib)
+    assert call(lh=host) == _lib.E_INVALID and "lse" in _err(lib)        # lse_host without lse_dev
+    assert call(ld=fake) == _lib.E_INVALID and "lse" in _err(lib)        # lse_dev without lse_host
+    assert call(hpc=0) == _lib.E_INVALID and "heads_per_chunk" in _err(lib)
+    assert call(mo=1) == _lib.E_INVALID and "map_offset" in _err(lib)
+    assert call(d=96) == _lib.E_UNSUPPORTED
+    assert call(dt=7) == _lib.E_UNSUPPORTED
+    assert call(qd=ctypes.c_void_p(0x10008)) == _lib.E_INVALID and "aligned" in _err(lib)
+    assert call(blp=None) == _lib.E_INVALID and "block list" in _err(lib)
+
+
 def test_workspace_queries(lib):
     n = ctypes.c_size_t(0)
     assert lib.calibatt_calibrate_workspace_size(40, 32760, 32768, 128, 128, 128, ctypes.byref(n)) == _lib.OK

@@ -93,6 +93,28 @@ def test_bf16_structured_scores():
     run_full_compare(q, k, v, mask, w.N, 128, "bf16", 128)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_large_score_jumps(d):
+    # Every query shares a direction u and every key carries u with a
+    # magnitude set per 64-key half block (32 levels in random order), so the
+    # running row maximum jumps by far more than the kernel's rescale
+    # threshold in first and second halves of blocks alike (a float64 walk of
+    # these inputs in the kernel's block order counts 11 / 22 such jumps at
+    # d = 128, 21 / 27 at d = 64): the redo and O-rescale paths run.
+    N, Np, H = 2000, 2048, 2
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 41)
+    rng = np.random.default_rng(42)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = (q + 8.0 * u).astype(np.float32)
+    g = 12.0 * np.repeat(rng.permutation(32), 64)
+    k = (k + g[None, None, :, None] * u).astype(np.float32)
+    mask = (rng.random((H, 16, 16)) < 0.5).astype(np.uint8)
+    mask[0, 5, :] = 1
+    mask[1, :, 15] = 1
+    run_full_compare(q, k, v, mask, N, 128, "bf16", d)
+
+
 def test_bf16_deterministic():
     N, Np, H = 1024, 1024, 2
     q, k, v = syn.normal_qkv(1, H, N, Np, 128, 21)
@@ -104,6 +126,33 @@ def test_bf16_deterministic():
     o1, l1 = cba.sparse_attn_fwd(qd, kd, vd, bl, N, return_lse=True)
     o2, l2 = cba.sparse_attn_fwd(qd, kd, vd, bl, N, return_lse=True)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("dtype,d,hpc", [("bf16", 128, 2), ("bf16", 64, 5), ("fp32", 64, 3)])
+def test_streamed_host_buffers_match_device_call(dtype, d, hpc):
+    # Same kernel per chunk of heads: the host-buffer call must reproduce the
+    # device call bit for bit, O and LSE, with a ragged last chunk and B = 2.
+    B, H, N, Np = 2, 5, 2000, 2048
+    q, k, v = syn.normal_qkv(B, H, N, Np, d, 51)
+    pair = bf16_pair if dtype == "bf16" else fp32_pair
+    _, qd = pair(q)
+    _, kd = pair(k)
+    _, vd = pair(v)
+    mask = (np.random.default_rng(6).random((H + 2, 16, 16)) < 0.4).astype(np.uint8)
+    mask[1, 3, :] = 0
+    bl = cba.compile(torch.from_numpy(mask).cuda())
+    o_ref, lse_ref = cba.sparse_attn_fwd(qd, kd, vd, bl, N, map_offset=1, return_lse=True)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (qd, kd, vd))
+    staging = (torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd),
+               torch.empty((B, H, Np), dtype=torch.float32, device="cuda"))
+    lse_h = torch.empty((B, H, Np), dtype=torch.float32).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o_h = cba.sparse_attn_fwd_streamed(qh, kh, vh, bl, N, staging, map_offset=1, heads_per_chunk=hpc, lse=lse_h,
+                                       status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(o_h, o_ref.cpu())
+    assert torch.equal(lse_h, lse_ref.cpu())
 
 
 def sampled_parity(w, mask, qkv=None, n_samples=24, seed=0, map_offset=0):
