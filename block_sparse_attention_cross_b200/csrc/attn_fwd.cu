@@ -6,29 +6,37 @@
 // kept-block list; only the kept K/V tiles are loaded (TMA) and multiplied
 // (tcgen05), so a skipped block costs neither bytes nor FLOPs.
 //
-// Persistent CTA (one per SM), 12 warps, two independent query-tile "slots":
-//   warps 0-3   softmax warpgroup of slot 0 (thread t owns row t = TMEM lane t)
-//   warps 4-7   softmax warpgroup of slot 1
-//   warp 8      TMA producer: Q tile per slot, K and V tiles of the kept blocks
+// Persistent CTA (one per SM, one query tile at a time), 12 warps:
+//   warps 0-3   softmax, key columns 0-63 of each block (warp w: rows 32w..32w+31)
+//   warps 4-7   softmax, key columns 64-127 of the same rows
+//   warp 8      TMA producer: the Q tile, then K and V tiles of the kept blocks
 //               into one shared ring, in exactly the order the MMA warp uses them
 //   warp 9      TMEM allocator and MMA issuer
 //   warps 10-11 idle (they complete the control warpgroup)
-// The block is launched with 168 registers per thread.  Inside its own branch
-// the control warpgroup lowers its limit to 56 and the softmax warpgroups
-// raise theirs to 224, which holds a full 128-column score row in registers:
-// 2 * 128 * 224 + 128 * 56 = 384 * 168.
-// The two slots have their own kept-block lists; while one slot's softmax
-// runs, the tensor core works on the other slot's QK^T and PV, so neither
-// waits for the other.  Per slot and block j the MMA issue order is
-// PV(j-1), S(j): S(j) overwrites the TMEM columns holding P(j-1), which the
-// in-order tensor pipe has already consumed.
+// The block is launched with 168 registers per thread; inside its own branch
+// the control warpgroup (two walk cursors per role) lowers its limit to 120
+// and the softmax warpgroups raise theirs to 192 (a 64-column half row of
+// scores in registers): 2 * 128 * 192 + 128 * 120 = 384 * 168.
 //
-// TMEM (512 columns): slot s uses [256 s, 256 s + 128) for S, overwritten in
-// place by P as bf16 pairs (the A operand of the PV MMA), and
-// [256 s + 128, 256 s + 128 + d) for the O accumulator.
-// Softmax: exp2 on the scaled scores; the running max is only raised (and O
-// rescaled in TMEM) when it grows by more than 8 (log2 units), which keeps
-// every P value <= 256 and O / l exact.
+// TMEM (512 columns): two score buffers S0 = [0, 128) and S1 = [128, 256) and
+// the O accumulator [256, 256 + d).  Block g of the CTA's walk uses buffer
+// g % 2.  The softmax half h overwrites the first 32 columns of its own 64
+// score columns with its probabilities as bf16 pairs, so P of one block sits
+// at columns [0, 32) and [64, 96) of its buffer: the A operand of the PV MMA
+// (tcgen05.mma with A in TMEM), issued as two K = 64 groups.
+// MMA issue order: S(0), S(1), then PV(g), S(g + 2) for g = 0, 1, ...: the
+// tensor core computes the scores of block g + 1 and PV of block g - 1 while
+// the softmax works on block g, and S(g + 2) may overwrite P(g) because the
+// in-order tensor pipe has consumed it.
+//
+// Softmax: exp2 of the scaled scores against a reference max m shared by the
+// two halves of a row.  The first block of a tile takes the exact row max
+// (the halves exchange their maxima through shared memory); later blocks are
+// exponentiated against the current m while their max is found, and the
+// halves exchange their block maxima after their stores are in flight.  Only
+// when a row's block max exceeds m by more than kRescaleThreshold is the
+// block redone with the raised m and O rescaled (after the previous PV has
+// completed).
 // Every wait is bounded; on expiry the CTA reports CALIBATT_E_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <cmath>
@@ -42,8 +50,8 @@ namespace {
 constexpr int TILE = 128;
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kSoftmaxRegs = 224;
-constexpr uint32_t kControlRegs = 56;
+constexpr uint32_t kSoftmaxRegs = 192;
+constexpr uint32_t kControlRegs = 120;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs, "register split");
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -64,9 +72,11 @@ struct FwdLayout {
   static constexpr uint32_t BOX_BYTES = TILE * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
   static constexpr uint32_t TILE_BYTES = TILE * D * 2;
   static constexpr int RING = (D == 128) ? 5 : 10;
-  static constexpr uint32_t OFF_Q = 0;                   // 2 slots
-  static constexpr uint32_t OFF_RING = 2 * TILE_BYTES;
-  static constexpr uint32_t OFF_CTRL = OFF_RING + RING * TILE_BYTES;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_RING = TILE_BYTES;
+  static constexpr uint32_t OFF_XCHG = OFF_RING + RING * TILE_BYTES;   // float2 [2 slots][2 halves][128 rows]
+  static constexpr uint32_t XCHG_BYTES = 2 * 2 * 128 * 8;
+  static constexpr uint32_t OFF_CTRL = OFF_XCHG + XCHG_BYTES;
   static constexpr uint32_t CTRL_BYTES = 1024;
   static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
 };
@@ -74,9 +84,11 @@ struct FwdLayout {
 template <int RING>
 struct FwdCtrl {
   uint64_t ring_full[RING], ring_empty[RING];
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2];
-  uint64_t o_full[2], o_free[2];
+  uint64_t pv_done;
+  uint64_t o_full, o_free;
+  uint64_t xchg[4];   // per row quarter: the two softmax warps of those rows
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -138,31 +150,54 @@ __device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool repor
   return tl;
 }
 
-// Static schedule shared by the producer and the MMA warp.  Slot s of CTA c
-// takes work tiles c + s*G, c + s*G + 2G, ... (G = gridDim.x), skipping
-// tiles with empty lists.  A step of a slot is "PV of the previous block (if
-// any), then QK^T of the next block (if any)".
-struct SlotSched {
-  int t, n, base, p0, bh, j, pv, rot;
+// Walk over the kept blocks of this CTA's non-empty work tiles c, c + G,
+// c + 2G, ... (G = gridDim.x), shared by the producer and the MMA warp.
+struct Cursor {
+  int t, n, base, p0, bh, qb, rot, j;
   bool done;
 };
 
-__device__ __forceinline__ void sched_next_tile(const TcArgs& a, SlotSched& st, int T, int stride) {
-  while (st.t < T) {
-    const TileList tl = tile_list(a, st.t, false);
+__device__ __forceinline__ void cursor_seek(const TcArgs& a, Cursor& cu, int T, int G) {
+  while (cu.t < T) {
+    const TileList tl = tile_list(a, cu.t, false);
     if (tl.n > 0) {
-      st.n = tl.n;
-      st.base = tl.base;
-      st.p0 = tl.p0;
-      st.bh = tl.bh;
-      st.rot = tl.rot;
-      st.j = 0;
-      st.pv = -1;
+      cu.n = tl.n;
+      cu.base = tl.base;
+      cu.p0 = tl.p0;
+      cu.bh = tl.bh;
+      cu.qb = tl.qb;
+      cu.rot = tl.rot;
+      cu.j = 0;
       return;
     }
-    st.t += stride;
+    cu.t += G;
   }
-  st.done = true;
+  cu.done = true;
+}
+
+__device__ __forceinline__ void cursor_init(const TcArgs& a, Cursor& cu, int T, int G) {
+  cu.t = blockIdx.x;
+  cu.done = false;
+  cursor_seek(a, cu, T, G);
+}
+
+__device__ __forceinline__ void cursor_next(const TcArgs& a, Cursor& cu, int T, int G) {
+  if (++cu.j == cu.n) {
+    cu.t += G;
+    cursor_seek(a, cu, T, G);
+  }
+}
+
+__device__ __forceinline__ int cursor_kb(const TcArgs& a, const Cursor& cu) {
+  return cu.base + a.pat_off[cu.p0 + (cu.j + cu.rot) % cu.n];
+}
+
+// The score stream (S, K tiles) runs up to two blocks ahead of the PV stream
+// (PV, V tiles): S(gs) reuses the buffer of block gs - 2, whose PV must have
+// been issued.  Producer and MMA warp take the same decision from their own
+// counters, so the ring is filled in exactly the order it is consumed.
+__device__ __forceinline__ bool take_score(const Cursor& cs, uint32_t gs, uint32_t gp) {
+  return !cs.done && gs <= gp + 1;
 }
 
 template <int D>
@@ -186,14 +221,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c->ring_full[e], 1);
       mbar_init(&c->ring_empty[e], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&c->q_full[s], 1);
-      mbar_init(&c->q_empty[s], 1);
-      mbar_init(&c->s_full[s], 1);
-      mbar_init(&c->p_full[s], 128);
-      mbar_init(&c->o_full[s], 1);
-      mbar_init(&c->o_free[s], 128);
+    mbar_init(&c->q_full, 1);
+    mbar_init(&c->q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&c->s_full[b], 1);
+      mbar_init(&c->p_full[b], 256);
     }
+    mbar_init(&c->pv_done, 1);
+    mbar_init(&c->o_full, 1);
+    mbar_init(&c->o_free, 256);
+    for (int w = 0; w < 4; ++w) mbar_init(&c->xchg[w], 64);
     mbar_init(&c->drain, 1);
     c->abort = 0;
     fence_barrier_init();
@@ -213,73 +250,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) regs_dec<kControlRegs>();
   if (warp == kProducerWarp) {
     // ===================== TMA producer =======================================
-    SlotSched st[2];
-    for (int s = 0; s < 2; ++s) {
-      st[s].t = blockIdx.x + s * G;
-      st[s].done = false;
-      sched_next_tile(a, st[s], T, 2 * G);
-    }
-    uint32_t g = 0;         // ring fills issued
-    int qfills[2] = {0, 0};
+    Cursor cs, cp;
+    cursor_init(a, cs, T, G);
+    cursor_init(a, cp, T, G);
+    uint32_t g = 0, gs = 0, gp = 0;   // ring fills, K tiles, V tiles issued
+    int qfills = 0;
     bool ok = true;
     const uint64_t pol = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
-    while (ok && !(st[0].done && st[1].done)) {
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
+    while (ok && !(cs.done && cp.done)) {
+      const bool score = take_score(cs, gs, gp);
+      if (score && cs.j == 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty, (qfills & 1) ^ 1, &c->abort, a.spin_ns));
         if (!ok) break;
-        SlotSched& q = st[s];
-        if (q.done) continue;
-        if (q.pv >= 0) {
-          const int kb = q.base + a.pat_off[q.p0 + (q.pv + q.rot) % q.n];
-          const int row = q.bh * a.Np + kb * TILE;
-          const int e = g % R;
-          ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
-          if (ok) {
-            mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
+        mbar_arrive_expect_tx_w(&c->q_full, L::TILE_BYTES);
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x)
-              tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, &tmV, x * 64, row,
-                            &c->ring_full[e], pol);
-          }
-          if (!ok) break;
-          ++g;
-          q.pv = -1;
-          if (q.j == q.n) {
-            q.t += 2 * G;
-            sched_next_tile(a, q, T, 2 * G);
-            if (q.done) continue;
-          }
-        }
-        const int j = q.j;
-        if (j == 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty[s], (qfills[s] & 1) ^ 1, &c->abort, a.spin_ns));
-          if (ok) {
-            const int qrow = q.bh * a.Np + (q.t % a.nqb) * TILE;
-            mbar_arrive_expect_tx_w(&c->q_full[s], L::TILE_BYTES);
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_2d_w(smem + L::OFF_Q + x * L::BOX_BYTES, &tmQ, x * 64, cs.bh * a.Np + cs.qb * TILE, &c->q_full,
+                        pol_q);
+        ++qfills;
+      }
+      const int row = score ? cs.bh * a.Np + cursor_kb(a, cs) * TILE : cp.bh * a.Np + cursor_kb(a, cp) * TILE;
+      const int e = g % R;
+      ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
+      if (!ok) break;
+      mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
+      const CUtensorMap* tm = score ? &tmK : &tmV;
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x)
-              tma_load_2d_w(smem + L::OFF_Q + s * L::TILE_BYTES + x * L::BOX_BYTES, &tmQ, x * 64, qrow,
-                            &c->q_full[s], pol_q);
-          }
-          if (!ok) break;
-          ++qfills[s];
-        }
-        const int kb = q.base + a.pat_off[q.p0 + (j + q.rot) % q.n];
-        const int row = q.bh * a.Np + kb * TILE;
-        const int e = g % R;
-        ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
-        if (ok) {
-          mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
-#pragma unroll
-          for (int x = 0; x < D / 64; ++x)
-            tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, &tmK, x * 64, row,
-                          &c->ring_full[e], pol);
-        }
-        if (!ok) break;
-        ++g;
-        q.pv = j;
-        q.j = j + 1;
+      for (int x = 0; x < D / 64; ++x)
+        tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, tm, x * 64, row, &c->ring_full[e],
+                      pol);
+      ++g;
+      if (score) {
+        ++gs;
+        cursor_next(a, cs, T, G);
+      } else {
+        ++gp;
+        cursor_next(a, cp, T, G);
       }
     }
     if (lane == 0) {
@@ -292,85 +299,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fills = (g > static_cast<uint32_t>(e)) ? (g - 1 - e) / R + 1 : 0;
         if (fills > 0) mbar_wait(&c->ring_full[e], (fills - 1) & 1, nullptr, a.spin_ns);
       }
-      for (int s = 0; s < 2; ++s)
-        if (qfills[s] > 0) mbar_wait(&c->q_full[s], (qfills[s] - 1) & 1, nullptr, a.spin_ns);
+      if (qfills > 0) mbar_wait(&c->q_full, (qfills - 1) & 1, nullptr, a.spin_ns);
     }
   } else if (warp == kMmaWarp) {
     // ===================== MMA issuer =========================================
-    SlotSched st[2];
-    for (int s = 0; s < 2; ++s) {
-      st[s].t = blockIdx.x + s * G;
-      st[s].done = false;
-      sched_next_tile(a, st[s], T, 2 * G);
-    }
+    Cursor cs, cp;
+    cursor_init(a, cs, T, G);
+    cursor_init(a, cp, T, G);
     constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false);
     constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
     const uint32_t sQ = smem_u32(smem + L::OFF_Q);
     const uint32_t sRing = smem_u32(smem + L::OFF_RING);
-    uint32_t g = 0;
-    int tiles[2] = {0, 0};   // tiles started per slot
-    int pvs[2] = {0, 0};     // PV MMAs issued per slot
+    const uint32_t tO = tmem + 256;
+    uint32_t g = 0, gs = 0, gp = 0;
+    int qtiles = 0;   // tiles whose first S was issued
+    int otiles = 0;   // tiles whose first PV was issued
     bool ok = true;
-    while (ok && !(st[0].done && st[1].done)) {
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        if (!ok) break;
-        SlotSched& q = st[s];
-        if (q.done) continue;
-        const uint32_t tS = tmem + s * 256;
-        const uint32_t tO = tS + 128;
-        if (q.pv >= 0) {
-          const int e = g % R;
-          ok = mbar_wait(&c->p_full[s], pvs[s] & 1, &c->abort, a.spin_ns) &&
-               mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns) &&
-               (q.pv > 0 || mbar_wait(&c->o_free[s], ((tiles[s] - 1) & 1) ^ 1, &c->abort, a.spin_ns));
-          ok = __all_sync(0xffffffffu, ok);
-          if (ok) {
-            tc_fence_after();
-            const uint32_t sV = sRing + e * L::TILE_BYTES;
-            mma_ts_k128_w(tO, tS, sdesc_sw128(sV, L::BOX_BYTES, 1024), IDESC_O, q.pv > 0 ? 1u : 0u);
-            mma_commit_w(&c->ring_empty[e]);
-            if (q.pv == q.n - 1) mma_commit_w(&c->o_full[s]);
-          }
-          if (!ok) break;
-          ++g;
-          ++pvs[s];
-          q.pv = -1;
-          if (q.j == q.n) {
-            q.t += 2 * G;
-            sched_next_tile(a, q, T, 2 * G);
-            if (q.done) continue;
-          }
-        }
-        const int j = q.j;
-        const int e = g % R;
-        if (j == 0) ++tiles[s];
-        ok = (j > 0 || mbar_wait(&c->q_full[s], (tiles[s] - 1) & 1, &c->abort, a.spin_ns)) &&
+    while (ok && !(cs.done && cp.done)) {
+      const int e = g % R;
+      if (take_score(cs, gs, gp)) {
+        const uint32_t tS = tmem + (gs & 1) * 128;
+        ok = (cs.j > 0 || mbar_wait(&c->q_full, qtiles & 1, &c->abort, a.spin_ns)) &&
              mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns);
         ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t sQs = sQ + s * L::TILE_BYTES;
-          const uint32_t sK = sRing + e * L::TILE_BYTES;
-          if (D == 128) {
-            mma_ss_k128_w(tS, sdesc_sw128(sQs, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::BOX_BYTES >> 4);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ad = sdesc_sw128(sQs + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
-              mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-            }
-          }
-          mma_commit_w(&c->s_full[s]);
-          mma_commit_w(&c->ring_empty[e]);
-          if (j == q.n - 1) mma_commit_w(&c->q_empty[s]);
-        }
         if (!ok) break;
-        ++g;
-        q.pv = j;
-        q.j = j + 1;
+        tc_fence_after();
+        const uint32_t sK = sRing + e * L::TILE_BYTES;
+        if (D == 128) {
+          mma_ss_k128_w(tS, sdesc_sw128(sQ, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::BOX_BYTES >> 4);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+            mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit_w(&c->s_full[gs & 1]);
+        mma_commit_w(&c->ring_empty[e]);
+        if (cs.j == 0) ++qtiles;
+        if (cs.j == cs.n - 1) mma_commit_w(&c->q_empty);
+        ++gs;
+        cursor_next(a, cs, T, G);
+      } else {
+        const uint32_t tP = tmem + (gp & 1) * 128;
+        ok = mbar_wait(&c->p_full[gp & 1], (gp >> 1) & 1, &c->abort, a.spin_ns) &&
+             mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns) &&
+             (cp.j > 0 || mbar_wait(&c->o_free, (otiles & 1) ^ 1, &c->abort, a.spin_ns));
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t vd = sdesc_sw128(sRing + e * L::TILE_BYTES, L::BOX_BYTES, 1024);
+        // keys 0-63 (P columns [0, 32)), then keys 64-127 (P columns [64, 96))
+        mma_ts_k64_w(tO, tP, vd, IDESC_O, cp.j > 0 ? 1u : 0u);
+        mma_ts_k64_w(tO, tP + 64, vd + 512, IDESC_O, 1u);
+        mma_commit_w(&c->ring_empty[e]);
+        mma_commit_w(&c->pv_done);
+        if (cp.j == 0) ++otiles;
+        if (cp.j == cp.n - 1) mma_commit_w(&c->o_full);
+        ++gp;
+        cursor_next(a, cp, T, G);
       }
+      ++g;
     }
     if (!ok && lane == 0) {
       c->abort = 1;
@@ -382,24 +372,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // ===================== softmax warpgroups =================================
     regs_inc<kSoftmaxRegs>();
-    const int s = warp >> 2;                  // slot
+    const int h = warp >> 2;                  // key-column half of every block
     const int w = warp & 3;                   // TMEM lane quarter
     const int row = w * 32 + lane;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(w * 32) << 16) + s * 256;
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(w * 32) << 16);
     const float c2 = a.scale_log2;
-    int sc = 0;      // S tiles consumed by this slot
-    int tiles = 0;   // non-empty tiles finished by this slot
+    float2* xbuf = reinterpret_cast<float2*>(smem + L::OFF_XCHG);
+    uint32_t xc = 0;   // exchanges with the partner warp (same rows, other half)
+    uint32_t gb = 0;   // blocks of non-empty tiles consumed by this CTA
+    int tiles = 0;     // non-empty tiles finished
     bool ok = true;
-    for (int t = blockIdx.x + s * G; ok && t < T; t += 2 * G) {
+    // Posts this thread's value for its row, then (finish) waits for the
+    // partner's; the two steps may be split to overlap other work.
+    auto xpost = [&](float2 v) {
+      xbuf[((xc & 1) * 2 + h) * 128 + row] = v;
+      mbar_arrive(&c->xchg[w]);
+    };
+    auto xfinish = [&]() -> float2 {
+      const bool got = mbar_wait(&c->xchg[w], xc & 1, &c->abort, a.spin_ns);
+      ok = __all_sync(0xffffffffu, got) && ok;
+      const float2 v = xbuf[((xc & 1) * 2 + (h ^ 1)) * 128 + row];
+      ++xc;
+      return v;
+    };
+    for (int t = blockIdx.x; ok && t < T; t += G) {
       const TileList tl = tile_list(a, t, true);
       const int grow = tl.qb * TILE + row;
       const size_t orow_idx = static_cast<size_t>(tl.bh) * a.Np + grow;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D + h * (D / 2);
       if (tl.n == 0) {
         uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = z;
-        if (a.lse != nullptr) a.lse[orow_idx] = -INFINITY;
+        for (int i = 0; i < D / 16; ++i) reinterpret_cast<uint4*>(orow)[i] = z;
+        if (a.lse != nullptr && h == 0) a.lse[orow_idx] = -INFINITY;
         continue;
       }
       const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
@@ -407,39 +412,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
       float m = -INFINITY;
       float l = 0.f;
-      // Largest raw score of the row so far (for the normalisation fix-up in
-      // the epilogue).
+      // Largest raw score of this half-row so far (for the normalisation
+      // fix-up in the epilogue).
       float s_best = -INFINITY;
-      for (int j = 0; j < tl.n; ++j) {
-        ok = mbar_wait(&c->s_full[s], sc & 1, &c->abort, a.spin_ns);
-        ok = __all_sync(0xffffffffu, ok);
+      for (int j = 0; j < tl.n; ++j, ++gb) {
+        const uint32_t b = gb & 1;
+        const bool got = mbar_wait(&c->s_full[b], (gb >> 1) & 1, &c->abort, a.spin_ns);
+        ok = __all_sync(0xffffffffu, got);
         if (!ok) break;
-        ++sc;
         tc_fence_after();
-        uint32_t r[TILE];
-#pragma unroll
-        for (int q4 = 0; q4 < TILE / 32; ++q4)
-          tmem_ld32(t_lane + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
+        const uint32_t t_s = t_row + b * 128 + h * 64;   // this half's 64 score columns
+        uint32_t r[64];
+        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_ld_wait();
         reg_fence(r);
         if (j == j_last && valid_last < TILE) {
           // Key columns past the sequence end exist only in the last block.
 #pragma unroll
-          for (int i = 0; i < TILE; ++i)
-            if (i >= valid_last) r[i] = f2u(-INFINITY);
+          for (int i = 0; i < 64; ++i)
+            if (h * 64 + i >= valid_last) r[i] = f2u(-INFINITY);
         }
-        // p = 2^(s c2 - mref) two columns at a time (pairs selected by kPolyFrom
-        // use the FMA-pipe polynomial, the rest the MUFU unit).  P (bf16 pairs)
-        // overwrites the first 64 columns of this slot's S region, 16 columns
-        // (32 probabilities) per store.  Returns the row sum; with `track` it
-        // also returns the row maximum of the raw scores.
+        // p = 2^(s c2 - mref) two columns at a time (pairs selected by
+        // kPolyFrom use the FMA-pipe polynomial, the rest the MUFU unit), as
+        // bf16 pairs into the first 32 columns of this half's score columns,
+        // 16 columns (32 probabilities) per store.  Returns the half-row sum;
+        // with `track` it also returns the half-row maximum of the raw scores.
         const uint64_t c2x2 = f2pack(c2, c2);
         auto emit_p = [&](float mref, bool track, float& mx_out) -> float {
           const uint64_t negm = f2pack(-mref, -mref);
           uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
           float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-          for (int c16 = 0; c16 < TILE / 32; ++c16) {
+          for (int c16 = 0; c16 < 2; ++c16) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -462,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               f2unpack(pv, pl, ph);
               pk[i] = pack_bf16x2(pl, ph);
             }
-            tmem_st16(t_lane + c16 * 16, pk);
+            tmem_st16(t_s + c16 * 16, pk);
           }
           mx_out = fmaxf(mxa, mxb);
           float a0, a1, b0, b1;
@@ -473,30 +478,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         float alpha = 1.f;
         float rs;
         if (j == 0) {
-          // First block of the tile: the exact row maximum sets the reference.
+          // First block of the tile: the exact row maximum (both halves) sets
+          // the reference.
           float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
 #pragma unroll
-          for (int i = 4; i < TILE; i += 8) {
+          for (int i = 4; i < 64; i += 8) {
             mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
             mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
             mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
             mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
           }
           s_best = fmax3(mx0, mx1, fmaxf(mx2, mx3));
-          m = s_best * c2;
+          xpost(make_float2(s_best, 0.f));
+          const float2 other = xfinish();
+          m = fmaxf(s_best, other.x) * c2;
           float unused;
           rs = emit_p(m, false, unused);
         } else {
           // Later blocks: exponentiate against the current reference while
-          // finding the block maximum.  Only if some row's maximum exceeds the
+          // finding the block maximum; the halves exchange their maxima while
+          // the stores are in flight.  Only if a row's maximum exceeds the
           // reference by more than the threshold (rare) is the block redone
           // with the raised reference and O rescaled.
           float mx;
           rs = emit_p(m, true, mx);
-          const float m_cand = mx * c2;
-          const bool raise = m_cand > m + kRescaleThreshold;
+          xpost(make_float2(mx, 0.f));
           s_best = fmaxf(s_best, mx);
+          const float m_cand = fmaxf(mx, xfinish().x) * c2;
+          const bool raise = m_cand > m + kRescaleThreshold;
           if (__any_sync(0xffffffffu, raise)) {
+            // O must hold PV of every earlier block of the tile: wait for the
+            // previous block's PV (the commit that signalled S(j) covers the
+            // ones before it).
+            const bool pv = mbar_wait(&c->pv_done, (gb - 1) & 1, &c->abort, a.spin_ns);
+            ok = __all_sync(0xffffffffu, pv) && ok;
+            tc_fence_after();
             if (raise) {
               alpha = ex2_approx(m - m_cand);
               m = m_cand;
@@ -504,50 +520,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();   // the speculative P stores land before they are overwritten
             float unused;
             rs = emit_p(m, false, unused);
-            // O holds PV(0..j-1) complete: the commit that signalled S(j)
-            // covers every MMA issued before it.
 #pragma unroll
-            for (int q4 = 0; q4 < D / 32; ++q4) {
+            for (int q4 = 0; q4 < D / 64; ++q4) {
               uint32_t ro[32];
-              tmem_ld32(t_lane + 128 + q4 * 32, ro);
+              const uint32_t t_o = t_row + 256 + h * (D / 2) + q4 * 32;
+              tmem_ld32(t_o, ro);
               tmem_ld_wait();
               reg_fence(ro);
 #pragma unroll
               for (int i = 0; i < 32; ++i) ro[i] = f2u(u2f(ro[i]) * alpha);
-              tmem_st32(t_lane + 128 + q4 * 32, ro);
+              tmem_st32(t_o, ro);
             }
           }
         }
         l = l * alpha + rs;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&c->p_full[s]);
+        mbar_arrive(&c->p_full[b]);
+        if (!ok) break;
       }
       if (!ok) break;
       // ---- epilogue: O / l, LSE -------------------------------------------
-      ok = mbar_wait(&c->o_full[s], tiles & 1, &c->abort, a.spin_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ++tiles;
-      tc_fence_after();
       // O holds sums of bf16-rounded probabilities while l sums the fp32 ones.
       // Their mismatch is negligible except for a dominant probability, which
       // is not exactly representable once the reference lags the row maximum
-      // (threshold above): its rounding error, recomputed here exactly as the
-      // softmax formed it, is moved into the normaliser so that a row with one
-      // dominant key returns that key's value.  The row's largest score was
-      // always exponentiated against the final reference m: a raise after its
-      // block would need a larger score, and a raise in its block redoes the
-      // block against that very score (p = 1, exact).  The LSE keeps the fp32
-      // sum.
+      // (threshold above): the rounding error of each half's largest
+      // probability, re-formed here exactly as the softmax formed it, is moved
+      // into the normaliser, so that a row with one dominant key returns that
+      // key's value.  The largest score was always exponentiated against the
+      // final reference m: a raise after its block would need a larger score,
+      // and a raise in its block redoes the block against a reference at or
+      // above it.  The LSE keeps the fp32 sum.
       const float p_best = ex2_approx(fmaf(s_best, c2, -m));
-      const float l_o = l + (__uint_as_float(pack_bf16x2(p_best, 0.f) << 16) - p_best);
+      const float corr = __uint_as_float(pack_bf16x2(p_best, 0.f) << 16) - p_best;
+      xpost(make_float2(l, corr));
+      const float2 other = xfinish();
+      const float l_row = l + other.x;
+      const float l_o = l_row + (corr + other.y);
+      const bool got = mbar_wait(&c->o_full, tiles & 1, &c->abort, a.spin_ns);
+      ok = __all_sync(0xffffffffu, got) && ok;
+      if (!ok) break;
+      ++tiles;
+      tc_fence_after();
       const bool pad_row = grow >= a.N;
       const float inv_l = pad_row ? 0.f : 1.f / l_o;
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) {
+      for (int q4 = 0; q4 < D / 64; ++q4) {
         uint32_t r[32];
-        tmem_ld32(t_lane + 128 + q4 * 32, r);
+        tmem_ld32(t_row + 256 + h * (D / 2) + q4 * 32, r);
         tmem_ld_wait();
         reg_fence(r);
         uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
@@ -562,8 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&c->o_free[s]);
-      if (a.lse != nullptr) a.lse[orow_idx] = pad_row ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+      mbar_arrive(&c->o_free);
+      if (a.lse != nullptr && h == 0)
+        a.lse[orow_idx] = pad_row ? -INFINITY : (m + log2f(l_row)) * 0.69314718055994531f;
     }
     if (!ok) {
       c->abort = 1;
@@ -608,7 +629,7 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
       return check_launch("cudaDeviceGetAttribute(SM count)");
   }
   const long long T = static_cast<long long>(a.B) * a.H * a.nqb;
-  const int grid = static_cast<int>(std::min<long long>(g_num_sms, (T + 1) / 2));
+  const int grid = static_cast<int>(std::min<long long>(g_num_sms, T));
   kern<<<grid, kThreads, FwdLayout<D>::SMEM_BYTES, s>>>(tq, tk, tv, a);
   count_launch();
   return check_launch("k_attn_fwd");
