@@ -131,3 +131,13 @@ def test_calibrate_wan_config_subset():
     assert np.array_equal(mask.cpu().numpy(), m_o)
     np.testing.assert_allclose(np.stack(Eg)[:, :, :, :].sum(axis=-1), 1.0, atol=2e-3)
     print(f"PARITY calibrate-wan480 8 inputs: votes and masks bit-exact; mask density {float(mask.float().mean()):.4f}")
+    # time of one calibration pass (8 inputs: energies, selection, votes, mask) on the device
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    cba.calibrate(qd, kd, w.N, select_param=0.25, rho=0.5)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    flops = I * 2 * 2 * w.N * w.N * w.d * w.H   # two QK^T passes per input
+    print(f"TIMING calibrate-wan480 8 inputs: {ms:.1f} ms, energy passes {flops / ms / 1e9:.1f} TFLOP/s")
