@@ -372,7 +372,8 @@ def main_calibatt(args):
     per_launch_ms = statistics.mean(per) / len(offsets)
     achieved = flops_step / len(offsets) / (per_launch_ms / 1e3) / 1e12
 
-    extras = {}
+    extras = {"step_ms_stats": {"median": round(statistics.median(per), 4), "min": round(min(per), 4),
+                                "max": round(max(per), 4), "steps": len(per)}}
     if sweep:
         # per-call time against density: one call per (layer, timestep)
         per, dens_call = [], []
@@ -403,6 +404,15 @@ def main_calibatt(args):
             dens_sweep.append({"density": round(b.density, 4), "ms": round(td / 20, 4),
                           "kept_tflops": round(kept_flops(b.nnz, w.d, w.B) / (td / 20 / 1e3) / 1e12, 1)})
         extras["density_sweep"] = dens_sweep
+        # wall time against kept fraction: linear fit, and kept-block throughput at 0.2 against 1.0
+        xd = np.asarray([r["density"] for r in dens_sweep])
+        yd = np.asarray([r["ms"] for r in dens_sweep])
+        sl, ic = np.polyfit(xd, yd, 1)
+        r2d = 1.0 - np.sum((yd - (sl * xd + ic)) ** 2) / np.sum((yd - yd.mean()) ** 2)
+        def at(d):
+            return min(dens_sweep, key=lambda r: abs(r["density"] - d))["kept_tflops"]
+        extras["density_fit"] = {"ms_per_unit_density": round(float(sl), 4), "intercept_ms": round(float(ic), 4),
+                                 "r2": round(float(r2d), 5), "kept_tflops_0.2_over_1.0": round(at(0.2) / at(1.0), 4)}
         # end to end through the public API with host buffers
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         ho = torch.empty_like(hq).pin_memory()

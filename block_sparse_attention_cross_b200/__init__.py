@@ -27,7 +27,7 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
                    CalibattError, check, load)
 
 __all__ = [
-    "BlockList", "sparse_attn_fwd", "block_energy", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",

@@ -141,3 +141,31 @@ def test_calibrate_wan_config_subset():
     ms = e0.elapsed_time(e1)
     flops = I * 2 * 2 * w.N * w.N * w.d * w.H   # two QK^T passes per input
     print(f"TIMING calibrate-wan480 8 inputs: {ms:.1f} ms, energy passes {flops / ms / 1e9:.1f} TFLOP/s")
+
+
+def test_sharded_calibration_single_rank_matches_calibrate():
+    # Calibration sharded by input, run as one NCCL rank on one GPU: the
+    # gather, per-input selection, votes and threshold must give exactly the
+    # single-call calibration's mask, votes and energy sums.
+    import os
+    import socket
+    import torch.distributed as dist
+    from block_sparse_attention_cross_b200.sharded import calibrate_sharded
+    H = 2
+    w, inputs = small_inputs(4, H, syn.VideoGrid(3, 20, 50), 128)
+    qd = [bf16_pair(q)[1] for q, _ in inputs]
+    kd = [bf16_pair(k)[1] for _, k in inputs]
+    mask1, votes1, esum1 = cba.calibrate(qd, kd, w.N, select_param=0.25, rho=0.5)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        mask2, votes2, esum2 = calibrate_sharded(qd, kd, w.N, select_param=0.25, rho=0.5)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert torch.equal(votes1, votes2)
+    assert torch.equal(esum1, esum2)
+    assert torch.equal(mask1, mask2)

@@ -63,3 +63,35 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
 
     bench.main_reference(A())
     assert capsys.readouterr().out == ""
+
+
+def _gather_worker(rank, world, port, out):
+    from block_sparse_attention_cross_b200.sharded import gather_in_order
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r holds inputs with ids; rank 0 two, rank 1 one, rank 2 three
+        counts = [2, 1, 3][:world]
+        first = sum(counts[:rank])
+        local = [torch.full((2, 3, 4), float(first + i)) + torch.arange(24.0).view(2, 3, 4) * 1e-3
+                 for i in range(counts[rank])]
+        got = gather_in_order(local)
+        out[rank] = [float(t[0, 0, 0]) for t in got] + [tuple(got[0].shape)]
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_calibration_gathers_inputs_in_global_order_gloo(world):
+    # The cross-rank step of calibration sharded by input: every rank must see
+    # every input's energies in global input order (rank-major), whatever the
+    # per-rank counts, so that selection, votes and the float32 energy sums
+    # replay the single-GPU order exactly.
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_gather_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+    n = sum([2, 1, 3][:world])
+    for rank in range(world):
+        assert out[rank][:-1] == [float(i) for i in range(n)]
+        assert out[rank][-1] == (2, 3, 4)
