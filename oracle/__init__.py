@@ -22,6 +22,9 @@ blocking, fusion or reordering beyond what the definition states):
   top key blocks (Figure 5(a); Figure S8 energy threshold).
 * ``vote``               -- agreement voting across calibration inputs
   (Figure 3(b) keep frequency; Figure 7 agreement threshold rho).
+* ``timestep_clusters`` / ``share_masks`` -- timestep sharing of calibrated
+  masks (Figure S11 skipped-block IoU across timesteps; Table S3 clusters of
+  pair-wise IoU >= tau).
 * ``compile_blocklist`` / ``expand_blocklist`` -- compile masks into per-row
   kept-block lists with translation-relative row-pattern dedup (Abstract:
   "compiles these patterns into optimized attention operations for each
@@ -38,6 +41,7 @@ for epsilon values, not for the selection rule).
 from .attention import masked_attention, masked_attention_rows, dense_attention_lse
 from .calibration import block_energy, select_topk, select_energy, topk_count, vote, min_votes_for
 from .compile import compile_blocklist, expand_blocklist
+from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
 
 __all__ = [
     "masked_attention",

@@ -325,3 +325,78 @@ def test_compile_empty_and_full():
     assert bl["n_pat"] == 1 and bl["nnz"] == 0 and bl["nnz_pat"] == 0
     bl = oracle.compile_blocklist(np.ones((2, 3, 4), np.uint8))
     assert bl["n_pat"] == 2 and bl["nnz_pat"] == 4 and np.all(bl["row_pat"] == 1) and np.all(bl["row_base"] == 0)
+
+
+# ---------------------------------------------------------------- O6 timestep sharing
+
+def test_skipped_iou_hand_cases():
+    # skipped sets {1, 2} and {2, 3}: intersection 1, union 3
+    assert oracle.skipped_iou([1, 0, 0, 1], [1, 1, 0, 0]) == pytest.approx(1 / 3)
+    assert oracle.skipped_iou([0, 1, 0], [0, 1, 0]) == 1.0
+    assert oracle.skipped_iou([0, 1, 1], [1, 0, 1]) == 0.0           # disjoint skipped sets
+    assert oracle.skipped_iou([1, 1], [1, 1]) == 1.0                 # nothing skipped: identical
+
+
+def test_skipped_iou_matches_set_arithmetic():
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        a = (rng.random(37) < 0.6).astype(np.uint8)
+        b = (rng.random(37) < 0.6).astype(np.uint8)
+        sa = {i for i in range(37) if a[i] == 0}
+        sb = {i for i in range(37) if b[i] == 0}
+        want = 1.0 if not (sa | sb) else len(sa & sb) / len(sa | sb)
+        assert oracle.skipped_iou(a, b) == want
+
+
+def _runs_masks():
+    # one layer, one head, 4 timesteps: t0 == t1, t2 == t3, t1 and t2 far apart
+    base = np.zeros((4, 4), np.uint8)
+    m0 = base.copy(); m0[0, :] = 1
+    m2 = base.copy(); m2[:, 3] = 1; m2[1, :] = 1
+    return np.stack([m0, m0, m2, m2])[None, :, None]
+
+
+def test_timestep_clusters_hand_case_and_extremes():
+    masks = _runs_masks()
+    assert oracle.timestep_clusters(masks, 0.9).tolist() == [[0, 0, 1, 1]]
+    assert oracle.timestep_clusters(masks, 0.0).tolist() == [[0, 0, 0, 0]]
+    assert oracle.timestep_clusters(masks, 1.01).tolist() == [[0, 1, 2, 3]]
+
+
+def test_timestep_clusters_are_pairwise_and_greedy():
+    rng = np.random.default_rng(11)
+    L, T, H = 3, 7, 2
+    base = rng.random((L, 1, H, 6, 6)) < 0.5
+    flips = rng.random((L, T, H, 6, 6)) < rng.choice([0.02, 0.1, 0.4], size=(L, T, 1, 1, 1))
+    masks = (base ^ np.cumsum(flips, axis=1).astype(bool)).astype(np.uint8)
+    for tau in (0.3, 0.6, 0.9):
+        cl = oracle.timestep_clusters(masks, tau)
+        for l in range(L):
+            ids = cl[l].tolist()
+            assert ids[0] == 0 and all(b - a in (0, 1) for a, b in zip(ids, ids[1:]))   # consecutive runs
+            for c in set(ids):
+                mem = [t for t in range(T) if ids[t] == c]
+                for t1 in mem:                                                          # pair-wise >= tau
+                    for t2 in mem:
+                        if t1 != t2:
+                            sim = np.mean([oracle.skipped_iou(masks[l, t1, h], masks[l, t2, h]) for h in range(H)])
+                            assert sim >= tau
+            for t in range(1, T):                                                       # greedy: a new run
+                if ids[t] != ids[t - 1]:                                                # had a reason to start
+                    prev = [s for s in range(t) if ids[s] == ids[t - 1]]
+                    sims = [np.mean([oracle.skipped_iou(masks[l, t, h], masks[l, s, h]) for h in range(H)])
+                            for s in prev]
+                    assert min(sims) < tau
+
+
+def test_share_masks_union_and_offsets():
+    masks = _runs_masks()
+    cl = oracle.timestep_clusters(masks, 0.9)
+    shared, off = oracle.share_masks(masks, cl)
+    assert shared.shape == (2, 1, 4, 4)
+    assert off.tolist() == [[0, 0, 1, 1]]
+    for t in range(4):
+        got = shared[off[0, t]]
+        assert np.all(got >= masks[0, t])                 # nothing a member keeps is skipped
+    singleton = oracle.share_masks(masks, np.array([[0, 1, 2, 3]]))[0]
+    assert np.array_equal(singleton[:, 0], masks[0, :, 0])
