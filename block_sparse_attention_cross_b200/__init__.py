@@ -27,7 +27,8 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
                    CalibattError, check, load)
 
 __all__ = [
-    "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
+    "share_masks", "share_timesteps", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -288,6 +289,52 @@ def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mo
                                         int(min_votes), _ptr(mask), _ptr(ws), ws.numel(), _ptr(status),
                                         _stream(dev)))
     return mask, votes, energy_sum
+
+
+def timestep_clusters(masks, tau):
+    """Runs of alike consecutive timesteps per layer (synchronizes).
+
+    ``masks``: uint8 [L, T, H, nqb, nkb] CUDA tensor.  Returns (run_of, n_runs):
+    run_of an int32 [L, T] CPU tensor of global run indices in (layer, time)
+    order, n_runs their number.
+    """
+    _need_cuda(masks)
+    if masks.dtype != torch.uint8 or masks.dim() != 5:
+        raise ValueError("masks must be uint8 [L, T, H, nqb, nkb]")
+    L, T, H, nqb, nkb = masks.shape
+    n = ctypes.c_size_t(0)
+    check(load().calibatt_timestep_clusters_workspace_size(L, T, H, ctypes.byref(n)))
+    ws = torch.empty(max(int(n.value), 1), dtype=torch.uint8, device=masks.device)
+    run_of = torch.empty((L, T), dtype=torch.int32)
+    n_runs = ctypes.c_int32(0)
+    with torch.cuda.device(masks.device):
+        check(load().calibatt_timestep_clusters(_ptr(masks), L, T, H, nqb, nkb, float(tau), _ptr(run_of),
+                                                ctypes.byref(n_runs), _ptr(ws), ws.numel(), _stream(masks.device)))
+    return run_of, n_runs.value
+
+
+def share_masks(masks, run_of, n_runs):
+    """Union masks [n_runs, H, nqb, nkb] uint8 of the runs ``run_of`` ([L, T] int32)."""
+    _need_cuda(masks)
+    L, T, H, nqb, nkb = masks.shape
+    run_dev = run_of.to(device=masks.device, dtype=torch.int32).contiguous()
+    shared = torch.empty((int(n_runs), H, nqb, nkb), dtype=torch.uint8, device=masks.device)
+    with torch.cuda.device(masks.device):
+        check(load().calibatt_share_masks(_ptr(masks), L, T, H, nqb, nkb, _ptr(run_dev), int(n_runs), _ptr(shared),
+                                          _stream(masks.device)))
+    return shared
+
+
+def share_timesteps(masks, tau):
+    """Timestep sharing of a [L, T, H, nqb, nkb] mask dictionary.
+
+    Returns (shared masks [n_runs * H, nqb, nkb] ready for :func:`compile`,
+    map_offset [L, T] int64 CPU tensor: the ``map_offset`` of call (l, t)).
+    """
+    run_of, n_runs = timestep_clusters(masks, tau)
+    shared = share_masks(masks, run_of, n_runs)
+    H = masks.shape[2]
+    return shared.reshape(n_runs * H, *masks.shape[3:]), run_of.to(torch.int64) * H
 
 
 def _compile_ws(n_maps, nqb, nkb, dev):

@@ -43,6 +43,11 @@ EXPORTS = {
                                                   c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
                                                   c_int, c_int, c_int, c_float, c_void_p, c_int, c_int, c_void_p,
                                                   c_void_p]),
+    "calibatt_timestep_clusters_workspace_size": (c_int, [c_int, c_int, c_int, POINTER(c_size_t)]),
+    "calibatt_timestep_clusters": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_double, c_void_p,
+                                           POINTER(c_int32), c_void_p, c_size_t, c_void_p]),
+    "calibatt_share_masks": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p,
+                                     c_void_p]),
     "calibatt_block_energy": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "calibatt_block_energy_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,

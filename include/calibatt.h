@@ -292,6 +292,45 @@ int calibatt_block_energy_noalloc(const void* q, const void* k, int H, int N, in
                                   int32_t* dev_status, calibatt_stream_t stream);
 
 /*
+ * calibatt_timestep_clusters -- groups the timesteps of every layer whose
+ * calibrated masks are alike, so that they can share one mask.
+ *
+ * Paper page, Figure S11 (IoU of the skipped-block masks of two timesteps,
+ * averaged over layers and heads; later, consecutive timesteps are alike) and
+ * Table S3 (timestep sharing clusters masks with pair-wise IoU >= tau).
+ * For layer l, the similarity of timesteps t1, t2 is the mean over heads h of
+ *     |S(l,t1,h) & S(l,t2,h)| / |S(l,t1,h) | S(l,t2,h)|,  S = blocks with mask 0
+ * (1 when both masks skip nothing).  Timesteps are grouped into runs of
+ * consecutive steps, greedily in time order: step t joins the current run
+ * when its similarity with every member is >= tau, otherwise it starts a new
+ * run.  Runs are numbered globally in (layer, time) order.
+ *  masks      [L, T, H, nqb, nkb] uint8 device (nonzero = kept; map order
+ *             (l T + t) H + h).
+ *  run_of     host int32 [L * T] (written): the run of every (l, t);
+ *  n_runs     host int32 (written): the number of runs.
+ *  workspace  device, >= calibatt_timestep_clusters_workspace_size bytes,
+ *             256-byte aligned.
+ * Synchronizes the stream (the grouping runs on the host from exact integer
+ * pair counts computed on the device).  T <= 1024.
+ */
+int calibatt_timestep_clusters_workspace_size(int L, int T, int H, size_t* bytes);
+int calibatt_timestep_clusters(const uint8_t* masks, int L, int T, int H, int nqb, int nkb, double tau,
+                               int32_t* run_of, int32_t* n_runs, void* workspace, size_t workspace_bytes,
+                               calibatt_stream_t stream);
+
+/*
+ * calibatt_share_masks -- one mask per run: the union of the kept blocks of
+ * the run's members (nothing any member keeps is skipped).
+ *  masks     [L, T, H, nqb, nkb] uint8 device;  run_of_dev device int32
+ *            [L * T] as returned by calibatt_timestep_clusters;
+ *  shared    [n_runs, H, nqb, nkb] uint8 device (written, 0/1).
+ * The call (l, t) then uses map_offset = run_of[l T + t] * H of the shared
+ * dictionary.  Asynchronous on `stream`.
+ */
+int calibatt_share_masks(const uint8_t* masks, int L, int T, int H, int nqb, int nkb, const int32_t* run_of_dev,
+                         int n_runs, uint8_t* shared, calibatt_stream_t stream);
+
+/*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the
  * bounded wait every kernel here uses, on a barrier that nothing completes.
  * After `limit_ns` it gives up and writes CALIBATT_E_TIMEOUT to dev_status.

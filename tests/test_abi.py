@@ -156,3 +156,22 @@ def test_binding_fails_loudly_without_cuda_tensors():
     x = torch.zeros(1, 1, 128, 64)
     with pytest.raises(ValueError):
         cba.sparse_attn_fwd(x, x, x, None, 128)
+
+
+def test_timestep_sharing_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    run = (ctypes.c_int32 * 8)()
+    n = ctypes.c_int32(0)
+    size = ctypes.c_size_t(0)
+    assert lib.calibatt_timestep_clusters_workspace_size(2, 4, 3, ctypes.byref(size)) == _lib.OK
+    assert size.value == 2 * 2 * 3 * 4 * 4 * 8
+    assert lib.calibatt_timestep_clusters(None, 2, 4, 3, 8, 8, 0.5, run, ctypes.byref(n), fake, size.value,
+                                          None) == _lib.E_INVALID
+    assert lib.calibatt_timestep_clusters(fake, 2, 2000, 3, 8, 8, 0.5, run, ctypes.byref(n), fake, 1 << 30,
+                                          None) == _lib.E_UNSUPPORTED
+    assert lib.calibatt_timestep_clusters(fake, 2, 4, 3, 8, 8, 0.5, run, ctypes.byref(n), fake, 16,
+                                          None) == _lib.E_WORKSPACE
+    assert lib.calibatt_timestep_clusters(fake, 2, 4, 3, 8, 8, float("nan"), run, ctypes.byref(n), fake,
+                                          size.value, None) == _lib.E_INVALID
+    assert lib.calibatt_share_masks(fake, 2, 4, 3, 8, 8, fake, 0, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_share_masks(fake, 2, 4, 3, 8, 8, fake, 9, fake, None) == _lib.E_INVALID
