@@ -19,11 +19,12 @@ pytestmark = pytest.mark.gpu
 
 
 def drifting_masks(L, T, H, nb, seed):
-    # masks that drift from step to step at a per-layer rate, so runs of
-    # several lengths appear
+    # masks whose kept blocks flip from step to step at a per-layer rate
+    # (1% ... 40%), so the layers split into runs of very different lengths
     rng = np.random.default_rng(seed)
     base = rng.random((L, 1, H, nb, nb)) < 0.4
-    flips = rng.random((L, T, H, nb, nb)) < rng.choice([0.005, 0.03, 0.2], size=(L, 1, 1, 1, 1))
+    rates = np.array([0.01, 0.05, 0.15, 0.4])[:L].reshape(L, 1, 1, 1, 1)
+    flips = rng.random((L, T, H, nb, nb)) < rates
     return (base ^ (np.cumsum(flips, axis=1) % 2).astype(bool)).astype(np.uint8)
 
 
