@@ -25,6 +25,8 @@ blocking, fusion or reordering beyond what the definition states):
 * ``timestep_clusters`` / ``share_masks`` -- timestep sharing of calibrated
   masks (Figure S11 skipped-block IoU across timesteps; Table S3 clusters of
   pair-wise IoU >= tau).
+* ``interval_counts`` / ``merge_masks`` / ``skiplist_bytes`` -- the pages'
+  interval skip-list storage (Figure S9, Figure S10, Table S3).
 * ``compile_blocklist`` / ``expand_blocklist`` -- compile masks into per-row
   kept-block lists with translation-relative row-pattern dedup (Abstract:
   "compiles these patterns into optimized attention operations for each
@@ -42,6 +44,7 @@ from .attention import masked_attention, masked_attention_rows, dense_attention_
 from .calibration import block_energy, select_topk, select_energy, topk_count, vote, min_votes_for
 from .compile import compile_blocklist, expand_blocklist
 from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
+from .skiplist import interval_counts, merge_row, merge_masks, nearest_rank, skiplist_bytes
 
 __all__ = [
     "masked_attention",

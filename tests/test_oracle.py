@@ -400,3 +400,65 @@ def test_share_masks_union_and_offsets():
         assert np.all(got >= masks[0, t])                 # nothing a member keeps is skipped
     singleton = oracle.share_masks(masks, np.array([[0, 1, 2, 3]]))[0]
     assert np.array_equal(singleton[:, 0], masks[0, :, 0])
+
+
+# ---------------------------------------------------------------- O7 interval skip lists
+
+def test_interval_counts_hand_and_brute_force():
+    rows = np.array([[[1, 1, 0, 1, 0, 0, 1], [0] * 7, [1] * 7, [1, 0, 1, 0, 1, 0, 1]]], np.uint8)
+    assert oracle.interval_counts(rows).tolist() == [[3, 0, 1, 4]]
+    rng = np.random.default_rng(2)
+    m = (rng.random((3, 5, 41)) < 0.5).astype(np.uint8)
+    want = [[sum(1 for i in range(41) if m[a, b, i] and (i == 0 or not m[a, b, i - 1])) for b in range(5)]
+            for a in range(3)]
+    assert oracle.interval_counts(m).tolist() == want
+
+
+def test_merge_row_hand_cases():
+    assert oracle.merge_row([1, 0, 1, 0, 0, 1], 2).tolist() == [1, 1, 1, 0, 0, 1]     # smallest gap first
+    assert oracle.merge_row([1, 0, 1, 0, 0, 1], 1).tolist() == [1] * 6
+    assert oracle.merge_row([0, 1, 0, 0, 1, 0, 0, 1, 0], 2).tolist() == [0, 1, 1, 1, 1, 0, 0, 1, 0]  # tie: leftmost
+    assert oracle.merge_row([0, 0, 0], 1).tolist() == [0, 0, 0]
+    assert oracle.merge_row([1, 0, 1], 5).tolist() == [1, 0, 1]
+
+
+def test_merge_row_invariants():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        n = int(rng.integers(1, 60))
+        row = (rng.random(n) < rng.random()).astype(np.uint8)
+        width = int(rng.integers(1, 8))
+        out = oracle.merge_row(row, width)
+        cnt = int(oracle.interval_counts(row[None, None])[0, 0])
+        cnt_out = int(oracle.interval_counts(out[None, None])[0, 0])
+        assert np.all(out >= row)
+        assert cnt_out == min(cnt, width) if cnt else cnt_out == 0
+        kept = np.nonzero(row)[0]
+        if kept.size:
+            assert not out[:kept[0]].any() and not out[kept[-1] + 1:].any()
+        # the gaps filled are the smallest ones
+        gaps = []
+        i = 0
+        while i < n:
+            if row[i] == 0 and 0 < i and kept.size and kept[0] < i < kept[-1]:
+                j = i
+                while row[j] == 0:
+                    j += 1
+                gaps.append((j - i, bool(out[i])))
+                i = j
+            else:
+                i += 1
+        filled = [g for g, f in gaps if f]
+        unfilled = [g for g, f in gaps if not f]
+        assert len(filled) == max(0, cnt - width)
+        if filled and unfilled:
+            assert max(filled) <= min(unfilled)
+
+
+def test_nearest_rank_and_skiplist_bytes():
+    assert oracle.nearest_rank([4, 1, 3, 2], 50) == 2
+    assert oracle.nearest_rank([4, 1, 3, 2], 100) == 4
+    assert oracle.nearest_rank(list(range(1, 21)), 95) == 19
+    counts = np.array([[1, 3], [2, 2]])        # two layers of one map with two rows each
+    b = oracle.skiplist_bytes(counts, 1, 5, pct=50)
+    assert b == {"full": 2 * 2 * 3 * 8, "trimmed": 2 * 3 * 8 + 2 * 2 * 8, "merged": 2 * 1 * 8 + 2 * 2 * 8}
