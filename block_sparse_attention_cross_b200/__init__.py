@@ -28,7 +28,7 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
 
 __all__ = [
     "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
-    "share_masks", "share_timesteps", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -335,6 +335,73 @@ def share_timesteps(masks, tau):
     shared = share_masks(masks, run_of, n_runs)
     H = masks.shape[2]
     return shared.reshape(n_runs * H, *masks.shape[3:]), run_of.to(torch.int64) * H
+
+
+def interval_counts(masks):
+    """int32 [n_maps, nqb]: kept-block intervals of every row of uint8 masks [n_maps, nqb, nkb]."""
+    _need_cuda(masks)
+    n_maps, nqb, nkb = masks.shape
+    counts = torch.empty((n_maps, nqb), dtype=torch.int32, device=masks.device)
+    with torch.cuda.device(masks.device):
+        check(load().calibatt_interval_counts(_ptr(masks), n_maps, nqb, nkb, _ptr(counts), _stream(masks.device)))
+    return counts
+
+
+def merge_intervals(masks, width_per_map):
+    """Merges, in place, every row of map i to at most width_per_map[i] intervals.
+
+    Returns the number of filled blocks (synchronizes)."""
+    _need_cuda(masks)
+    n_maps, nqb, nkb = masks.shape
+    width = torch.as_tensor(width_per_map, dtype=torch.int32).to(masks.device).contiguous()
+    filled = torch.zeros(1, dtype=torch.int64, device=masks.device)
+    with torch.cuda.device(masks.device):
+        check(load().calibatt_merge_intervals(_ptr(masks), n_maps, nqb, nkb, _ptr(width), _ptr(filled),
+                                              _stream(masks.device)))
+    return int(filled.item())
+
+
+def skiplist_report(masks, maps_per_layer, pcts=(100.0, 99.0, 95.0)):
+    """Storage of a mask dictionary [n_maps, nqb, nkb] in the paper page's
+    padded per-layer interval skip lists (one interval = an int32 pair) next
+    to this library's compiled forms.
+
+    Per layer: full allocation (ceil(nkb / 2) intervals per row), trimmed to
+    the widest row, and merged at each percentile in ``pcts`` (nearest rank of
+    the layer's interval counts; outlier rows merged by
+    :func:`merge_intervals`, whose filled blocks lower the sparsity).  Host
+    arithmetic on the device's interval counts; synchronizes.
+    """
+    n_maps, nqb, nkb = masks.shape
+    counts = interval_counts(masks).cpu()
+    if n_maps % maps_per_layer:
+        raise ValueError("n_maps must be a multiple of maps_per_layer")
+    layers = n_maps // maps_per_layer
+    rows_per_layer = maps_per_layer * nqb
+    per_layer = counts.view(layers, rows_per_layer).to(torch.int64)
+    full = layers * rows_per_layer * ((nkb + 1) // 2) * 8
+    trimmed = int(per_layer.max(dim=1).values.sum()) * rows_per_layer * 8
+    kept = int((masks != 0).sum())
+    out = {"rows": n_maps * nqb, "kept_blocks": kept, "density": kept / float(n_maps * nqb * nkb),
+           "intervals_max": int(counts.max()), "intervals_p95": _nearest_rank(counts, 95.0),
+           "skiplist_full_bytes": full, "skiplist_trimmed_bytes": trimmed, "merged": []}
+    for pct in pcts:
+        widths = [_nearest_rank(per_layer[l], pct) for l in range(layers)]
+        m = masks.clone()
+        filled = merge_intervals(m, [w for w in widths for _ in range(maps_per_layer)])
+        out["merged"].append({"pct": pct, "bytes": sum(widths) * rows_per_layer * 8, "filled_blocks": filled,
+                              "density": (kept + filled) / float(n_maps * nqb * nkb)})
+        del m
+    nnz, n_pat, nnz_pat = compile_size(masks)
+    out["csr_bytes"] = (n_maps * nqb + 1) * 8 + nnz * 2
+    out["pattern_pool_bytes"] = n_maps * nqb * 8 + (n_pat + 1) * 4 + nnz_pat * 2
+    return out
+
+
+def _nearest_rank(values, pct):
+    v = torch.sort(values.reshape(-1).to(torch.int64)).values
+    k = max(1, math.ceil(pct / 100.0 * v.numel()))
+    return int(v[k - 1])
 
 
 def _compile_ws(n_maps, nqb, nkb, dev):

@@ -48,6 +48,8 @@ EXPORTS = {
                                            POINTER(c_int32), c_void_p, c_size_t, c_void_p]),
     "calibatt_share_masks": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p,
                                      c_void_p]),
+    "calibatt_interval_counts": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
+    "calibatt_merge_intervals": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "calibatt_block_energy": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "calibatt_block_energy_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,

@@ -331,6 +331,30 @@ int calibatt_share_masks(const uint8_t* masks, int L, int T, int H, int nqb, int
                          int n_runs, uint8_t* shared, calibatt_stream_t stream);
 
 /*
+ * calibatt_interval_counts -- the number of intervals (maximal runs of
+ * consecutive kept key blocks) of every row of a mask dictionary: the row
+ * length of the paper page's interval skip lists (Figure S9, Figure S10).
+ *  masks   [n_maps, nqb, nkb] uint8 device (nonzero = kept);
+ *  counts  [n_maps * nqb] int32 device (written).  Asynchronous.
+ */
+int calibatt_interval_counts(const uint8_t* masks, int n_maps, int nqb, int nkb, int32_t* counts,
+                             calibatt_stream_t stream);
+
+/*
+ * calibatt_merge_intervals -- merges outlier rows (paper page, Figure S10 (c)
+ * and Table S3): every row of map i with more than width[i] intervals has
+ * its smallest gaps (runs of skipped blocks between two kept blocks; ties to
+ * the leftmost gap) filled until width[i] intervals remain.  Filled blocks
+ * become kept (they are computed; the mask loses that much sparsity).
+ *  masks   [n_maps, nqb, nkb] uint8 device, modified in place; nkb <= 2048.
+ *  width   [n_maps] int32 device (values below 1 count as 1).
+ *  filled  one uint64 on the device: the number of filled blocks is added.
+ * Asynchronous.
+ */
+int calibatt_merge_intervals(uint8_t* masks, int n_maps, int nqb, int nkb, const int32_t* width,
+                             unsigned long long* filled, calibatt_stream_t stream);
+
+/*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the
  * bounded wait every kernel here uses, on a barrier that nothing completes.
  * After `limit_ns` it gives up and writes CALIBATT_E_TIMEOUT to dev_status.

@@ -175,3 +175,11 @@ def test_timestep_sharing_validation(lib):
                                           size.value, None) == _lib.E_INVALID
     assert lib.calibatt_share_masks(fake, 2, 4, 3, 8, 8, fake, 0, fake, None) == _lib.E_INVALID
     assert lib.calibatt_share_masks(fake, 2, 4, 3, 8, 8, fake, 9, fake, None) == _lib.E_INVALID
+
+
+def test_skiplist_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.calibatt_interval_counts(None, 2, 8, 8, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_interval_counts(fake, 0, 8, 8, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_merge_intervals(fake, 2, 8, 8, None, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_merge_intervals(fake, 2, 8, 4096, fake, fake, None) == _lib.E_UNSUPPORTED
