@@ -57,10 +57,12 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true", help="skip the density sweep, e2e and CPU baseline")
     p.add_argument("--heads", type=int, default=None,
                    help="use only the first H heads (a smaller case for profiling; default: all 40)")
-    p.add_argument("--workload", default=WORKLOAD, choices=["wan480_25", "wan720_20", "mochi_20", "sweep"],
+    p.add_argument("--workload", default=WORKLOAD,
+                   choices=["wan480_25", "wan720_20", "mochi_20", "sweep", "wan480_25_k64"],
                    help="wan480_25 (default, Wan 2.1 480p call, 25%% kept); wan720_20 / mochi_20 (20%% kept); "
                         "sweep (40 layers x 3 timesteps x 40 heads of the 480p shape, one step = 120 calls, "
-                        "per-map density 0.1-0.6)")
+                        "per-map density 0.1-0.6); wan480_25_k64 (the 480p call with 128 x 64 blocks, 25%% of "
+                        "the 64-key blocks kept; no extras)")
     return p.parse_args()
 
 
@@ -98,8 +100,13 @@ def weak_scaling_tflops(world, flops_per_rank_step, steps, t_max_ms):
     return world * flops_per_rank_step * steps / (t_max_ms / 1e3) / 1e12
 
 
-def kept_flops(nnz_blocks, d, B, block=128):
-    return 4.0 * block * block * d * B * nnz_blocks
+def kept_flops(nnz_blocks, d, B, block=128, block_k=None):
+    return 4.0 * block * (block if block_k is None else block_k) * d * B * nnz_blocks
+
+
+def key_block(name):
+    """Key-block size of a bench workload: the _k64 variants use 64-key blocks."""
+    return 64 if name.endswith("_k64") else 128
 
 
 def peaks():
@@ -196,7 +203,7 @@ SWEEP_LAYERS, SWEEP_STEPS = 40, 3
 def workload(heads=None, name=WORKLOAD):
     import dataclasses
     from block_sparse_attention_cross_b200 import synthetic as syn
-    w = syn.WORKLOADS["wan480_25" if name == "sweep" else name]
+    w = syn.WORKLOADS["wan480_25" if name == "sweep" else name.replace("_k64", "")]
     return dataclasses.replace(w, H=heads) if heads else w
 
 
@@ -213,6 +220,12 @@ def build_workload(device, heads=None, density=None, name=WORKLOAD):
     del q, k, v
     if name == "sweep":
         mask = torch.from_numpy(syn.sweep_masks(w, SWEEP_LAYERS, SWEEP_STEPS)).to(device)
+    elif key_block(name) == 64:
+        # structured 128-key mask, refined to 64-key blocks at the target density
+        dens = w.density if density is None else density
+        coarse = syn.workload_mask(w, density=min(1.0, 1.5 * dens))
+        mask = torch.from_numpy(syn.refine_key_blocks(coarse, dens, w.seeds.get("mask", 0) + 1)).to(device)
+        return w, tensors, cba.compile(mask, block_q=128, block_k=64)
     else:
         mask = torch.from_numpy(syn.workload_mask(w, density=density)).to(device)
     bl = cba.compile(mask)
@@ -297,9 +310,11 @@ def workload_label(name, w, bl):
         return (f"sweep: {SWEEP_LAYERS} layers x {SWEEP_STEPS} timesteps x {w.H} heads of the Wan-2.1-14B 480p "
                 f"shape ({shape} = {w.N} tokens, padded {w.Np}, d={w.d}, bf16, 128x128 blocks), one step = "
                 f"{SWEEP_LAYERS * SWEEP_STEPS} calls, per-map density U(0.1, 0.6), mean {100 * bl.density:.1f}% kept")
-    model = {"wan480_25": "Wan-2.1-14B 480p", "wan720_20": "Wan-2.1-14B 720p", "mochi_20": "Mochi-1"}[name]
+    model = {"wan480_25": "Wan-2.1-14B 480p", "wan720_20": "Wan-2.1-14B 720p", "mochi_20": "Mochi-1"}[
+        name.replace("_k64", "")]
+    blocks = "128x64 blocks" if key_block(name) == 64 else "128x128 blocks"
     return (f"{name}: {model}-shaped attention call, {shape} = {w.N} tokens (padded {w.Np}), {w.H} heads, "
-            f"d={w.d}, bf16, 128x128 blocks, {100 * bl.density:.1f}% of blocks kept (structured mask)")
+            f"d={w.d}, bf16, {blocks}, {100 * bl.density:.1f}% of blocks kept (structured mask)")
 
 
 def time_calls(fn, steps, warmup, torch, dist=None):
@@ -348,8 +363,11 @@ def main_calibatt(args):
     w, (q, k, v), bl = build_workload(dev, args.heads, name=args.workload)
     out = torch.empty_like(q)
     pk = peaks()
-    flops_step = kept_flops(bl.nnz, w.d, w.B)
+    bk = key_block(args.workload)
+    flops_step = kept_flops(bl.nnz, w.d, w.B, block_k=bk)
     sweep = args.workload == "sweep"
+    if bk != 128:
+        args.no_extras = True   # the extras (full mask, density sweep, e2e, oracle sample) use 128-key blocks
     offsets = [(l * SWEEP_STEPS + t) * w.H for l in range(SWEEP_LAYERS) for t in range(SWEEP_STEPS)] if sweep else [0]
 
     def step():
@@ -450,7 +468,7 @@ def main_calibatt(args):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_sustained"],
                          "unit": UNIT, "frac": round(achieved / pk["bf16_sustained"], 4),
                          "traffic": kernel_traffic(),
-                         "kernel": "k_attn_fwd<128>",
+                         "kernel": f"k_attn_fwd<{w.d}, {bk}>",
                          "peak_kind": f"bf16_tflops_sustained ({pk['source']}); burst {pk['bf16_burst']}",
                          "algorithmic_flops_per_launch": flops_step / len(offsets)},
             "gpu_launches": int(launches),

@@ -73,12 +73,12 @@ void load_encode() {
 }
 }  // namespace
 
-int make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols) {
+int make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   std::call_once(g_encode_once, load_encode);
   if (g_encode == nullptr) return set_error(CALIBATT_E_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -161,9 +161,9 @@ int check_fwd(const void* q, const void* k, const void* v, const void* o, int B,
   if (static_cast<long long>(B) * H * Np >= (1ll << 31))
     return set_error(CALIBATT_E_UNSUPPORTED, "B*H*Np must be below 2^31 rows");
   if (dtype == CALIBATT_BF16) {
-    if (!(d == 64 || d == 128) || bl->block_q != 128 || bl->block_k != 128)
-      return set_error(CALIBATT_E_UNSUPPORTED, "bf16 path supports d in {64,128} with 128x128 blocks");
-    if (nkb > 1024) return set_error(CALIBATT_E_UNSUPPORTED, "at most 1024 key blocks per row");
+    if (!(d == 64 || d == 128) || bl->block_q != 128 || !(bl->block_k == 128 || bl->block_k == 64))
+      return set_error(CALIBATT_E_UNSUPPORTED, "bf16 path supports d in {64,128} with 128x128 or 128x64 blocks");
+    if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
     return CALIBATT_OK;
   }
   if (dtype == CALIBATT_FP32) {
@@ -245,6 +245,7 @@ int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
     a.scale_log2 = scale * 1.4426950408889634f;
     a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
     a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
+    a.kscale = 128 / bl->block_k;
     a.o = o; a.lse = lse; a.status = dev_status; a.spin_ns = spin_limit_ns();
     return launch_tc_fwd(q, k, v, d, a, s);
   }

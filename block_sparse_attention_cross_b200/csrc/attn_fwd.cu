@@ -67,14 +67,17 @@ constexpr float kRescaleThreshold = 64.0f;
 // while the polynomial is off.
 constexpr int kPolyFrom = 8;
 
-template <int D>
+// D: head dim; BK: key-block size (128 or 64; query blocks are always 128).
+template <int D, int BK>
 struct FwdLayout {
-  static constexpr uint32_t BOX_BYTES = TILE * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
-  static constexpr uint32_t TILE_BYTES = TILE * D * 2;
-  static constexpr int RING = (D == 128) ? 5 : 10;
+  static constexpr uint32_t QBOX_BYTES = TILE * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle span)
+  static constexpr uint32_t KBOX_BYTES = BK * 64 * 2;    // BK rows x 64 bf16
+  static constexpr uint32_t Q_BYTES = TILE * D * 2;
+  static constexpr uint32_t KV_BYTES = BK * D * 2;
+  static constexpr int RING = ((D == 128) ? 5 : 10) * (TILE / BK);
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_RING = TILE_BYTES;
-  static constexpr uint32_t OFF_XCHG = OFF_RING + RING * TILE_BYTES;   // float2 [2 slots][2 halves][128 rows]
+  static constexpr uint32_t OFF_RING = Q_BYTES;
+  static constexpr uint32_t OFF_XCHG = OFF_RING + RING * KV_BYTES;   // float2 [2 slots][2 halves][128 rows]
   static constexpr uint32_t XCHG_BYTES = 2 * 2 * 128 * 8;
   static constexpr uint32_t OFF_CTRL = OFF_XCHG + XCHG_BYTES;
   static constexpr uint32_t CTRL_BYTES = 1024;
@@ -108,7 +111,7 @@ struct TileList {
 // Reads and checks the kept-block list of work tile t.  Warp-collective: every
 // lane returns the same result, and every role evaluates the same data, so
 // all roles agree on n.
-__device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool report) {
+__device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool report, int kscale) {
   TileList tl;
   tl.bh = t / a.nqb;
   tl.qb = t - tl.bh * a.nqb;
@@ -144,7 +147,7 @@ __device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool repor
   int below = 0;
   for (int i0 = 0; i0 < tl.n; i0 += 32) {
     const int i = i0 + lane;
-    below += __popc(__ballot_sync(0xffffffffu, i < tl.n && tl.base + a.pat_off[p0 + i] < tl.qb));
+    below += __popc(__ballot_sync(0xffffffffu, i < tl.n && tl.base + a.pat_off[p0 + i] < tl.qb * kscale));
   }
   tl.rot = (below < tl.n) ? below : 0;
   return tl;
@@ -159,7 +162,7 @@ struct Cursor {
 
 __device__ __forceinline__ void cursor_seek(const TcArgs& a, Cursor& cu, int T, int G) {
   while (cu.t < T) {
-    const TileList tl = tile_list(a, cu.t, false);
+    const TileList tl = tile_list(a, cu.t, false, a.kscale);
     if (tl.n > 0) {
       cu.n = tl.n;
       cu.base = tl.base;
@@ -200,12 +203,13 @@ __device__ __forceinline__ bool take_score(const Cursor& cs, uint32_t gs, uint32
   return !cs.done && gs <= gp + 1;
 }
 
-template <int D>
+template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, BK>;
   constexpr int R = L::RING;
+  constexpr int HB = BK / 2;   // key columns per softmax half
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FwdCtrl<R>* c = reinterpret_cast<FwdCtrl<R>*>(smem + L::OFF_CTRL);
@@ -263,22 +267,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (score && cs.j == 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty, (qfills & 1) ^ 1, &c->abort, a.spin_ns));
         if (!ok) break;
-        mbar_arrive_expect_tx_w(&c->q_full, L::TILE_BYTES);
+        mbar_arrive_expect_tx_w(&c->q_full, L::Q_BYTES);
 #pragma unroll
         for (int x = 0; x < D / 64; ++x)
-          tma_load_2d_w(smem + L::OFF_Q + x * L::BOX_BYTES, &tmQ, x * 64, cs.bh * a.Np + cs.qb * TILE, &c->q_full,
+          tma_load_2d_w(smem + L::OFF_Q + x * L::QBOX_BYTES, &tmQ, x * 64, cs.bh * a.Np + cs.qb * TILE, &c->q_full,
                         pol_q);
         ++qfills;
       }
-      const int row = score ? cs.bh * a.Np + cursor_kb(a, cs) * TILE : cp.bh * a.Np + cursor_kb(a, cp) * TILE;
+      const int row = score ? cs.bh * a.Np + cursor_kb(a, cs) * BK : cp.bh * a.Np + cursor_kb(a, cp) * BK;
       const int e = g % R;
       ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
       if (!ok) break;
-      mbar_arrive_expect_tx_w(&c->ring_full[e], L::TILE_BYTES);
+      mbar_arrive_expect_tx_w(&c->ring_full[e], L::KV_BYTES);
       const CUtensorMap* tm = score ? &tmK : &tmV;
 #pragma unroll
       for (int x = 0; x < D / 64; ++x)
-        tma_load_2d_w(smem + L::OFF_RING + e * L::TILE_BYTES + x * L::BOX_BYTES, tm, x * 64, row, &c->ring_full[e],
+        tma_load_2d_w(smem + L::OFF_RING + e * L::KV_BYTES + x * L::KBOX_BYTES, tm, x * 64, row, &c->ring_full[e],
                       pol);
       ++g;
       if (score) {
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor cs, cp;
     cursor_init(a, cs, T, G);
     cursor_init(a, cp, T, G);
-    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, TILE, false);
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, BK, false);
     constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
     const uint32_t sQ = smem_u32(smem + L::OFF_Q);
     const uint32_t sRing = smem_u32(smem + L::OFF_RING);
@@ -324,14 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sK = sRing + e * L::TILE_BYTES;
-        if (D == 128) {
-          mma_ss_k128_w(tS, sdesc_sw128(sQ, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::BOX_BYTES >> 4);
+        const uint32_t sK = sRing + e * L::KV_BYTES;
+        if (D == 128 && BK == TILE) {
+          mma_ss_k128_w(tS, sdesc_sw128(sQ, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::QBOX_BYTES >> 4);
         } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32, 16, 1024);
+            const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32, 16, 1024);
             mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
         }
@@ -349,10 +353,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t vd = sdesc_sw128(sRing + e * L::TILE_BYTES, L::BOX_BYTES, 1024);
-        // keys 0-63 (P columns [0, 32)), then keys 64-127 (P columns [64, 96))
-        mma_ts_k64_w(tO, tP, vd, IDESC_O, cp.j > 0 ? 1u : 0u);
-        mma_ts_k64_w(tO, tP + 64, vd + 512, IDESC_O, 1u);
+        const uint64_t vd = sdesc_sw128(sRing + e * L::KV_BYTES, L::KBOX_BYTES, 1024);
+        if (BK == TILE) {
+          // keys 0-63 (P columns [0, 32)), then keys 64-127 (P columns [64, 96))
+          mma_ts_k64_w(tO, tP, vd, IDESC_O, cp.j > 0 ? 1u : 0u);
+          mma_ts_k64_w(tO, tP + 64, vd + 512, IDESC_O, 1u);
+        } else {
+          // half h's keys at P columns [h HB, h HB + HB / 2); 16 keys (8 columns,
+          // 16 V rows = 2048 bytes) per step
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const int hh = kk / (HB / 16), ks = kk % (HB / 16);
+            mma_bf16_ts_w(tO, tP + hh * HB + ks * 8, vd + kk * 128, IDESC_O, (cp.j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
         mma_commit_w(&c->ring_empty[e]);
         mma_commit_w(&c->pv_done);
         if (cp.j == 0) ++otiles;
@@ -396,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return v;
     };
     for (int t = blockIdx.x; ok && t < T; t += G) {
-      const TileList tl = tile_list(a, t, true);
+      const TileList tl = tile_list(a, t, true, TILE / BK);
       const int grow = tl.qb * TILE + row;
       const size_t orow_idx = static_cast<size_t>(tl.bh) * a.Np + grow;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D + h * (D / 2);
@@ -408,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
-      const int valid_last = (kb_last == a.nkb - 1) ? (a.N - kb_last * TILE) : TILE;
+      const int valid_last = (kb_last == a.nkb - 1) ? (a.N - kb_last * BK) : BK;
       const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
       float m = -INFINITY;
       float l = 0.f;
@@ -421,17 +435,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, got);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t t_s = t_row + b * 128 + h * 64;   // this half's 64 score columns
-        uint32_t r[64];
-        tmem_ld32(t_s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        const uint32_t t_s = t_row + b * 128 + h * HB;   // this half's HB score columns
+        uint32_t r[HB];
+#pragma unroll
+        for (int q4 = 0; q4 < HB / 32; ++q4)
+          tmem_ld32(t_s + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
         tmem_ld_wait();
         reg_fence(r);
-        if (j == j_last && valid_last < TILE) {
+        if (j == j_last && valid_last < BK) {
           // Key columns past the sequence end exist only in the last block.
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (h * 64 + i >= valid_last) r[i] = f2u(-INFINITY);
+          for (int i = 0; i < HB; ++i)
+            if (h * HB + i >= valid_last) r[i] = f2u(-INFINITY);
         }
         // p = 2^(s c2 - mref) two columns at a time (pairs selected by
         // kPolyFrom use the FMA-pipe polynomial, the rest the MUFU unit), as
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
           float mxa = -INFINITY, mxb = -INFINITY;
 #pragma unroll
-          for (int c16 = 0; c16 < 2; ++c16) {
+          for (int c16 = 0; c16 < HB / 32; ++c16) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -482,12 +497,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the reference.
           float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
 #pragma unroll
-          for (int i = 4; i < 64; i += 8) {
+          for (int i = 4; i + 8 <= HB; i += 8) {
             mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
             mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
             mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
             mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
           }
+          static_assert(HB % 8 == 0, "the loop above leaves exactly the last 4 columns");
+          mx0 = fmax3(mx0, u2f(r[HB - 4]), u2f(r[HB - 3]));
+          mx1 = fmax3(mx1, u2f(r[HB - 2]), u2f(r[HB - 1]));
           s_best = fmax3(mx0, mx1, fmaxf(mx2, mx3));
           xpost(make_float2(s_best, 0.f));
           const float2 other = xfinish();
@@ -600,14 +618,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int g_num_sms = 0;
 
-template <int D>
+template <int D, int BK>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
                cudaStream_t s) {
-  auto kern = k_attn_fwd<D>;
+  auto kern = k_attn_fwd<D, BK>;
+  constexpr uint32_t smem_bytes = FwdLayout<D, BK>::SMEM_BYTES;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<D>::SMEM_BYTES) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(k_attn_fwd)");
     configured = true;
   }
@@ -630,7 +648,7 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   }
   const long long T = static_cast<long long>(a.B) * a.H * a.nqb;
   const int grid = static_cast<int>(std::min<long long>(g_num_sms, T));
-  kern<<<grid, kThreads, FwdLayout<D>::SMEM_BYTES, s>>>(tq, tk, tv, a);
+  kern<<<grid, kThreads, smem_bytes, s>>>(tq, tk, tv, a);
   count_launch();
   return check_launch("k_attn_fwd");
 }
@@ -640,12 +658,13 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcArgs& a, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const uint64_t rows = static_cast<uint64_t>(a.B) * a.H * a.Np;
+  const uint32_t bk = static_cast<uint32_t>(TILE / a.kscale);   // key-block size: 128 or 64
   int rc;
-  if ((rc = make_tmap_bf16(&tq, q, rows, d)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tk, k, rows, d)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tv, v, rows, d)) != CALIBATT_OK) return rc;
-  if (d == 128) return launch_fwd<128>(tq, tk, tv, a, s);
-  return launch_fwd<64>(tq, tk, tv, a, s);
+  if ((rc = make_tmap_bf16(&tq, q, rows, d, TILE)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, rows, d, bk)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, rows, d, bk)) != CALIBATT_OK) return rc;
+  if (bk == 64) return d == 128 ? launch_fwd<128, 64>(tq, tk, tv, a, s) : launch_fwd<64, 64>(tq, tk, tv, a, s);
+  return d == 128 ? launch_fwd<128, 128>(tq, tk, tv, a, s) : launch_fwd<64, 128>(tq, tk, tv, a, s);
 }
 
 }  // namespace calibatt

@@ -25,6 +25,7 @@ struct TcArgs {
   const int32_t* pat_ptr;
   const int16_t* pat_off;
   int n_pat, nnz_pat, map_offset;
+  int kscale;              // forward: 128 / key-block size (1 or 2)
   void* o;                 // bf16 [B, H, Np, d]
   float* lse;              // [B, H, Np] natural-log LSE or nullptr
   float* lse2;             // calibration: per-row log2-domain LSE [H * Np]
@@ -69,7 +70,7 @@ int run_compile(const uint8_t* masks, int n_maps, int nqb, int nkb, int dedup, v
 // selftest
 int launch_selftest_timeout(uint64_t limit_ns, int32_t* status, cudaStream_t s);
 
-// TMA descriptor for a row-major bf16 matrix [rows, cols]; box 64 cols x 128 rows, 128-byte swizzle.
-int make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols);
+// TMA descriptor for a row-major bf16 matrix [rows, cols]; box 64 cols x box_rows rows, 128-byte swizzle.
+int make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows = 128);
 
 }  // namespace calibatt

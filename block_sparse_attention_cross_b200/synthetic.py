@@ -313,6 +313,34 @@ def workload_mask(w: Workload, density=None, n_maps=None, seed=None):
                                  block=w.block, period=period, forced_cols=forced)
 
 
+def refine_key_blocks(mask, density, seed):
+    """A mask on a key grid twice as fine (key blocks of 64 for query blocks of
+    128): each kept 128-key block contributes its two 64-key halves, both
+    halves of the query's own (diagonal) block are always kept, and the other
+    halves are kept at random to hit round(density * nqb * 2 nkb) exactly.
+    ``mask`` [n_maps, nqb, nkb] should keep more than ``density`` of its
+    blocks.  Returns uint8 [n_maps, nqb, 2 nkb].
+    """
+    rng = np.random.default_rng(seed)
+    n_maps, nqb, nkb = mask.shape
+    out = np.zeros((n_maps, nqb, 2 * nkb), dtype=np.uint8)
+    for m in range(n_maps):
+        cand = np.repeat(mask[m] != 0, 2, axis=1)
+        diag = np.zeros_like(cand)
+        q = np.arange(nqb)
+        diag[q, np.minimum(2 * q, 2 * nkb - 1)] = True
+        diag[q, np.minimum(2 * q + 1, 2 * nkb - 1)] = True
+        target = int(round(density * nqb * 2 * nkb))
+        keep = diag.copy()
+        rest = np.flatnonzero(cand & ~diag)
+        need = max(0, target - int(keep.sum()))
+        if need > rest.size:
+            raise ValueError("the coarse mask keeps too few blocks for this density")
+        keep.ravel()[rng.choice(rest, size=need, replace=False)] = True
+        out[m] = keep
+    return out
+
+
 def sweep_masks(w: Workload, layers=40, timesteps=3, seed=1000, lo=0.1, hi=0.6):
     """Mask dictionary of a denoising-step sweep: one structured mask per (layer, timestep, head).
 

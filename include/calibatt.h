@@ -129,8 +129,9 @@ uint64_t calibatt_get_spin_limit_ns(void);
  *           and n_q_blocks = n_k_blocks = Np / block_q;
  *           map_offset + H <= bl->n_maps.  The mask is shared by the batch.
  *  dev_status optional device int32 (see conventions).
- * Supported: CALIBATT_BF16 with d in {64, 128}, block 128 (tcgen05 tensor
- * cores, fp32 accumulation, P rounded to bf16 for the PV product);
+ * Supported: CALIBATT_BF16 with d in {64, 128}, block_q = 128 and block_k
+ * in {128, 64} (tcgen05 tensor cores, fp32 accumulation, P rounded to bf16
+ * for the PV product; paper page, Table S6 compares key-block sizes);
  * CALIBATT_FP32 with d in {64, 128}, block in {64, 128} (FFMA).  Anything
  * else returns CALIBATT_E_UNSUPPORTED.
  */

@@ -259,3 +259,80 @@ def test_bf16_sweep_dictionary_calls_sampled():
         err = np.concatenate(errs)
         assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (layer, t, err.max(), err.mean())
         print(f"PARITY sweep layer={layer} t={t} heads={w.H} max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
+
+
+def run_k64_compare(q, k, v, mask, N, d):
+    """Whole-tensor parity with 128-row query blocks and 64-key blocks."""
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    v64, vd = bf16_pair(v)
+    bl = cba.compile(torch.from_numpy(mask).cuda(), block_q=128, block_k=64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = cba.default_scale(d)
+    o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, N, scale=scale, return_lse=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    O, L = oracle.masked_attention(q64, k64, v64, mask, N, 128, 64, scale)
+    mx, mn = assert_close(to_np64(o), O, BF16_MAX_ABS, BF16_MEAN_ABS)
+    assert_lse(lse.cpu().numpy(), L, 1e-3)
+    print(f"PARITY bf16 128x64 blocks N={N} d={d} max_abs={mx:.3e} mean_abs={mn:.3e}")
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_key_blocks_of_64(d):
+    # 128-row query blocks with 64-key blocks: random masks with an empty row,
+    # a full row and the padded last key block kept everywhere, ragged N.
+    N, Np, H = 2000, 2048, 3
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 61)
+    rng = np.random.default_rng(62)
+    mask = (rng.random((H, 16, 32)) < 0.4).astype(np.uint8)
+    mask[0, 4, :] = 0
+    mask[1, 7, :] = 1
+    mask[2, :, 31] = 1
+    run_k64_compare(q, k, v, mask, N, d)
+
+
+def test_bf16_key_blocks_of_64_large_score_jumps():
+    # The redo / O-rescale paths with 64-key blocks (magnitudes set per
+    # 32-key quarter block, so jumps fall in both halves of a block).
+    N, Np, H, d = 2000, 2048, 2, 128
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 41)
+    rng = np.random.default_rng(43)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = (q + 8.0 * u).astype(np.float32)
+    g = 12.0 * np.repeat(rng.permutation(64), 32)
+    k = (k + g[None, None, :, None] * u).astype(np.float32)
+    mask = (rng.random((H, 16, 32)) < 0.5).astype(np.uint8)
+    mask[0, 5, :] = 1
+    run_k64_compare(q, k, v, mask, N, d)
+
+
+@pytest.mark.slow
+def test_bf16_key_blocks_of_64_wan480_sampled():
+    w = syn.WORKLOADS["wan480_25"]
+    coarse = syn.workload_mask(w, density=0.375)
+    mask = syn.refine_key_blocks(coarse, 0.25, 15)
+    q, k, v = syn.video_qkv(w)
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    v64, vd = bf16_pair(v)
+    del q, k, v
+    bl = cba.compile(torch.from_numpy(mask).cuda(), block_q=128, block_k=64)
+    assert bl.nnz == int(mask.sum())
+    scale = cba.default_scale(w.d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, w.N, scale=scale, return_lse=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rng = np.random.default_rng(16)
+    errs = []
+    for h, qb in [(0, 0), (w.H - 1, w.nqb - 1)] + [(int(rng.integers(w.H)), int(rng.integers(w.nqb)))
+                                                   for _ in range(14)]:
+        O, L = oracle.masked_attention_rows(q64, k64, v64, mask, w.N, 128, 64, scale, 0, h, qb)
+        rows = slice(qb * 128, (qb + 1) * 128)
+        errs.append(np.abs(to_np64(o[0, h, rows]) - O).ravel())
+        assert_lse(lse[0, h, rows].cpu().numpy(), L, 1e-3)
+    err = np.concatenate(errs)
+    assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
+    print(f"PARITY wan480 128x64 blocks sampled 16 query blocks max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
