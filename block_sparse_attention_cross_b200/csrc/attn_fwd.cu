@@ -6,6 +6,11 @@
 // kept-block list; only the kept K/V tiles are loaded (TMA) and multiplied
 // (tcgen05), so a skipped block costs neither bytes nor FLOPs.
 //
+// Templated on the head dim D (128 or 64) and the key-block size BK (128 or
+// 64; query blocks are always 128 rows; the paper page's Table S6 compares
+// key-block sizes).  The text below describes BK = 128; with BK = 64 every
+// key-column count halves (64-row K/V tiles, 32 columns per softmax half).
+//
 // Persistent CTA (one per SM, one query tile at a time), 12 warps:
 //   warps 0-3   softmax, key columns 0-63 of each block (warp w: rows 32w..32w+31)
 //   warps 4-7   softmax, key columns 64-127 of the same rows
