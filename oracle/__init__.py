@@ -27,6 +27,9 @@ blocking, fusion or reordering beyond what the definition states):
   pair-wise IoU >= tau).
 * ``interval_counts`` / ``merge_masks`` / ``skiplist_bytes`` -- the pages'
   interval skip-list storage (Figure S9, Figure S10, Table S3).
+* ``anchor_rows`` / ``anchor_attention`` -- spatial repetition: attention of
+  k anchor rows per frame broadcast to the other rows (Figure 4, Figure 5(b)
+  bottom, Table S4).
 * ``compile_blocklist`` / ``expand_blocklist`` -- compile masks into per-row
   kept-block lists with translation-relative row-pattern dedup (Abstract:
   "compiles these patterns into optimized attention operations for each
@@ -45,6 +48,7 @@ from .calibration import block_energy, select_topk, select_energy, topk_count, v
 from .compile import compile_blocklist, expand_blocklist
 from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
 from .skiplist import interval_counts, merge_row, merge_masks, nearest_rank, skiplist_bytes
+from .anchor import anchor_rows, anchor_attention
 
 __all__ = [
     "masked_attention",

@@ -462,3 +462,44 @@ def test_nearest_rank_and_skiplist_bytes():
     counts = np.array([[1, 3], [2, 2]])        # two layers of one map with two rows each
     b = oracle.skiplist_bytes(counts, 1, 5, pct=50)
     assert b == {"full": 2 * 2 * 3 * 8, "trimmed": 2 * 3 * 8 + 2 * 2 * 8, "merged": 2 * 1 * 8 + 2 * 2 * 8}
+
+
+# ---------------------------------------------------------------- O8 spatial repetition
+
+def test_anchor_rows_match_table_s4_row_sparsity_and_nearest():
+    import json
+    from pathlib import Path
+    g = json.loads((Path(__file__).parent / "golden" / "geometry.json").read_text())["table_s4_anchor_rows"]
+    for k, pct in zip(g["k"], g["sparsity_pct"]):
+        anchors, nearest = oracle.anchor_rows(30, k)
+        assert len(set(anchors)) == k
+        assert round(100.0 * (1 - len(set(anchors)) / 30), 1) == pct
+        for r in range(30):                        # nearest by brute force, ties to the lower anchor
+            dists = sorted((abs(a - r), a) for a in anchors)
+            assert nearest[r] == dists[0][1]
+    assert oracle.anchor_rows(30, 4)[0] == [3, 11, 18, 26]
+    assert oracle.anchor_rows(30, 4)[1][7] == 3     # |7-3| == |11-7|: the lower anchor
+    assert oracle.anchor_rows(12, 12) == (list(range(12)), list(range(12)))
+
+
+def test_anchor_attention_against_sdpa():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(21)
+    frames, rows, cols, d = 2, 6, 5, 16
+    N = frames * rows * cols
+    Np = N + 4
+    q, k, v = (rng.standard_normal((1, 2, Np, d)) for _ in range(3))
+    scale = 0.3
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[:, :, :N]), torch.from_numpy(k[:, :, :N]), torch.from_numpy(v[:, :, :N]),
+        scale=scale).numpy()
+    full = oracle.anchor_attention(q, k, v, N, frames, rows, cols, rows, scale)   # every row an anchor
+    assert np.allclose(full[:, :, :N], ref, atol=1e-12) and not full[:, :, N:].any()
+    o = oracle.anchor_attention(q, k, v, N, frames, rows, cols, 2, scale)
+    anchors, nearest = oracle.anchor_rows(rows, 2)
+    for f in range(frames):
+        for r in range(rows):
+            for c in range(cols):
+                t = f * rows * cols + r * cols + c
+                ta = f * rows * cols + nearest[r] * cols + c
+                assert np.allclose(o[:, :, t], ref[:, :, ta], atol=1e-12)
