@@ -20,6 +20,7 @@ import ctypes
 import math
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -28,7 +29,8 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
 
 __all__ = [
     "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
-    "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "gather_rows",
+    "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -195,6 +197,82 @@ def sparse_attn_fwd_streamed(q, k, v, bl: BlockList, N, staging, scale=None, map
             B, H, int(N), Np, d, _dtype_code(q), scale, ctypes.byref(s), int(map_offset), int(heads_per_chunk),
             _ptr(status), _stream(qd.device)))
     return out
+
+
+def gather_rows(src, idx, rows_dst=None):
+    """dst[..., i, :] = src[..., idx[i], :] over the leading dimensions (negative index: zero row)."""
+    _need_cuda(src)
+    idx_d = torch.as_tensor(idx, dtype=torch.int32).to(src.device).contiguous()
+    rows_dst = idx_d.numel() if rows_dst is None else rows_dst
+    lead = src.shape[:-2]
+    planes = int(np.prod(lead)) if len(lead) else 1
+    dst = torch.empty(tuple(lead) + (rows_dst, src.shape[-1]), dtype=src.dtype, device=src.device)
+    row_bytes = src.shape[-1] * src.element_size()
+    with torch.cuda.device(src.device):
+        check(load().calibatt_gather_rows(_ptr(src), _ptr(dst), _ptr(idx_d), planes, src.shape[-2], rows_dst,
+                                          row_bytes, _stream(src.device)))
+    return dst
+
+
+def anchor_rows(rows, k):
+    """The k anchor rows of a frame of ``rows`` spatial rows, evenly spaced and
+    centred, and for every row the anchor it takes its output from (the
+    nearest, the lower one on a tie)."""
+    anchors = [int(math.floor((i + 0.5) * rows / k)) for i in range(k)]
+    nearest = [min(anchors, key=lambda a: (abs(a - r), a)) for r in range(rows)]
+    return anchors, nearest
+
+
+@dataclass
+class AnchorPlan:
+    """Index lists of the spatial-repetition path for one video geometry."""
+    N: int
+    Np: int
+    nq: int          # gathered anchor query tokens
+    npq: int         # padded to a multiple of 128
+    idx_q: torch.Tensor   # [npq] int32: source token of every gathered query (-1: padding)
+    idx_o: torch.Tensor   # [Np] int32: gathered row every token's output comes from (-1: padding)
+
+
+def anchor_plan(frames, rows, cols, k_anchor, Np, device):
+    """Plan of :func:`anchor_attention` for a frames x rows x cols video padded to Np tokens."""
+    N = frames * rows * cols
+    anchors, nearest = anchor_rows(rows, k_anchor)
+    slot = {a: i for i, a in enumerate(anchors)}
+    fr = rows * cols
+    idx_q = [f * fr + a * cols + c for f in range(frames) for a in anchors for c in range(cols)]
+    nq = len(idx_q)
+    npq = (nq + 127) // 128 * 128
+    per_frame = len(anchors) * cols
+    idx_o = [f * per_frame + slot[nearest[r]] * cols + c for f in range(frames) for r in range(rows) for c in range(cols)]
+    as_dev = lambda x: torch.tensor(x, dtype=torch.int32, device=device)
+    return AnchorPlan(N, Np, nq, npq, as_dev(idx_q + [-1] * (npq - nq)), as_dev(idx_o + [-1] * (Np - N)))
+
+
+def anchor_attention(q, k, v, plan: AnchorPlan, bl=None, scale=None):
+    """Spatial-repetition attention (paper page, Figure 4, Figure 5(b) bottom,
+    Table S4): attention is computed only for the query tokens of the plan's
+    anchor rows (k evenly spaced spatial rows per frame) against all keys, and
+    every token takes the output of the token in the same frame and column on
+    its nearest anchor row.
+
+    q, k, v: [B, H, Np, d] bf16 CUDA tensors.  ``bl``: block list over the
+    gathered queries (n_q_blocks = plan.npq / 128, n_k_blocks = Np / block_k);
+    dense (every key block) when None.  Returns O [B, H, Np, d].
+    """
+    _need_cuda(q, k, v)
+    B, H, Np, d = q.shape
+    qg = gather_rows(q, plan.idx_q)
+    if bl is None:
+        bl = compile(torch.ones((H, plan.npq // 128, Np // 128), dtype=torch.uint8, device=q.device))
+    scale = default_scale(d) if scale is None else float(scale)
+    og = torch.empty_like(qg)
+    s = bl.as_struct()
+    with torch.cuda.device(q.device):
+        check(load().calibatt_sparse_attn_fwd_qk(_ptr(qg), _ptr(k), _ptr(v), _ptr(og), None, B, H, plan.nq, plan.npq,
+                                                 int(plan.N), Np, d, _dtype_code(q), scale, ctypes.byref(s), 0, None,
+                                                 _stream(q.device)))
+    return gather_rows(og, plan.idx_o)
 
 
 def _calib_workspace(H, N, Np, d, bq, bk, device):

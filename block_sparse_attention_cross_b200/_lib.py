@@ -50,6 +50,10 @@ EXPORTS = {
                                      c_void_p]),
     "calibatt_interval_counts": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]),
     "calibatt_merge_intervals": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "calibatt_sparse_attn_fwd_qk": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+                                            c_int, c_int, c_int, c_int, c_int, c_float, c_void_p, c_int, c_void_p,
+                                            c_void_p]),
+    "calibatt_gather_rows": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p]),
     "calibatt_block_energy": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                                       c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "calibatt_block_energy_noalloc": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,

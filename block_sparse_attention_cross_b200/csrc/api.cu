@@ -136,29 +136,32 @@ int validate_blocklist(const calibatt_blocklist* bl) {
 
 namespace {
 
-// Argument checks of the forward, shared by the plain and the streamed entry
-// points so that neither enqueues anything for a call it would reject.
-int check_fwd(const void* q, const void* k, const void* v, const void* o, int B, int H, int N, int Np, int d,
-              int dtype, float scale, const calibatt_blocklist* bl, int map_offset) {
+// Argument checks of the forward, shared by the plain, the streamed and the
+// gathered-query entry points so that none enqueues anything for a call it
+// would reject.  Queries have Nq real rows padded to Npq, keys Nk padded to Npk.
+int check_fwd(const void* q, const void* k, const void* v, const void* o, int B, int H, int Nq, int Npq, int Nk,
+              int Npk, int d, int dtype, float scale, const calibatt_blocklist* bl, int map_offset) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
     return set_error(CALIBATT_E_INVALID, "q, k, v and o must be non-NULL");
-  if (B <= 0 || H <= 0 || N <= 0 || Np < N || d <= 0)
-    return set_error(CALIBATT_E_INVALID, "bad sizes B=%d H=%d N=%d Np=%d d=%d", B, H, N, Np, d);
+  if (B <= 0 || H <= 0 || Nq <= 0 || Npq < Nq || Nk <= 0 || Npk < Nk || d <= 0)
+    return set_error(CALIBATT_E_INVALID, "bad sizes B=%d H=%d Nq=%d Npq=%d Nk=%d Npk=%d d=%d", B, H, Nq, Npq, Nk, Npk,
+                     d);
   if (!(scale > 0.f) || !std::isfinite(scale)) return set_error(CALIBATT_E_INVALID, "scale must be finite and > 0");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return set_error(CALIBATT_E_INVALID, "q, k, v, o must be 16-byte aligned");
   int rc = validate_blocklist(bl);
   if (rc) return rc;
-  if (bl->block_q <= 0 || bl->block_k <= 0 || Np % bl->block_q != 0 || Np % bl->block_k != 0)
-    return set_error(CALIBATT_E_INVALID, "Np=%d is not a multiple of the block sizes", Np);
-  const int nqb = Np / bl->block_q, nkb = Np / bl->block_k;
+  if (bl->block_q <= 0 || bl->block_k <= 0 || Npq % bl->block_q != 0 || Npk % bl->block_k != 0)
+    return set_error(CALIBATT_E_INVALID, "Np=%d/%d is not a multiple of the block sizes", Npq, Npk);
+  const int nqb = Npq / bl->block_q, nkb = Npk / bl->block_k;
   if (bl->n_q_blocks != nqb || bl->n_k_blocks != nkb)
     return set_error(CALIBATT_E_INVALID, "block list grid %dx%d does not match Np/block = %dx%d", bl->n_q_blocks,
                      bl->n_k_blocks, nqb, nkb);
-  if ((Np - N) >= bl->block_k) return set_error(CALIBATT_E_INVALID, "Np - N must be smaller than one block");
+  if ((Npk - Nk) >= bl->block_k || (Npq - Nq) >= bl->block_q)
+    return set_error(CALIBATT_E_INVALID, "Np - N must be smaller than one block");
   if (map_offset < 0 || static_cast<long long>(map_offset) + H > bl->n_maps)
     return set_error(CALIBATT_E_INVALID, "map_offset %d + H %d exceeds n_maps %d", map_offset, H, bl->n_maps);
-  if (static_cast<long long>(B) * H * Np >= (1ll << 31))
+  if (static_cast<long long>(B) * H * (Npq > Npk ? Npq : Npk) >= (1ll << 31))
     return set_error(CALIBATT_E_UNSUPPORTED, "B*H*Np must be below 2^31 rows");
   if (dtype == CALIBATT_BF16) {
     if (!(d == 64 || d == 128) || bl->block_q != 128 || !(bl->block_k == 128 || bl->block_k == 64))
@@ -167,6 +170,7 @@ int check_fwd(const void* q, const void* k, const void* v, const void* o, int B,
     return CALIBATT_OK;
   }
   if (dtype == CALIBATT_FP32) {
+    if (Nq != Nk || Npq != Npk) return set_error(CALIBATT_E_UNSUPPORTED, "fp32 path needs equal query and key lengths");
     if (!(d == 64 || d == 128) || !(bl->block_q == 64 || bl->block_q == 128) ||
         !(bl->block_k == 64 || bl->block_k == 128))
       return set_error(CALIBATT_E_UNSUPPORTED, "fp32 path supports d in {64,128}, blocks in {64,128}");
@@ -174,6 +178,32 @@ int check_fwd(const void* q, const void* k, const void* v, const void* o, int B,
     return CALIBATT_OK;
   }
   return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
+}
+
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Npq, int Nk,
+             int Npk, int d, int dtype, float scale, const calibatt_blocklist* bl, int map_offset, int32_t* dev_status,
+             calibatt_stream_t stream) {
+  int rc = check_fwd(q, k, v, o, B, H, Nq, Npq, Nk, Npk, d, dtype, scale, bl, map_offset);
+  if (rc) return rc;
+  const int nqb = Npq / bl->block_q, nkb = Npk / bl->block_k;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == CALIBATT_BF16) {
+    TcArgs a{};
+    a.B = B; a.H = H; a.N = Nq; a.Np = Npq; a.Nk = Nk; a.Npk = Npk; a.nqb = nqb; a.nkb = nkb;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
+    a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
+    a.kscale = 128 / bl->block_k;
+    a.o = o; a.lse = lse; a.status = dev_status; a.spin_ns = spin_limit_ns();
+    return launch_tc_fwd(q, k, v, d, a, s);
+  }
+  SimtArgs a{};
+  a.B = B; a.H = H; a.N = Nq; a.Np = Npq; a.block_q = bl->block_q; a.block_k = bl->block_k;
+  a.nqb = nqb; a.nkb = nkb; a.scale = scale;
+  a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
+  a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
+  a.lse = lse; a.status = dev_status;
+  return launch_simt_fwd(q, k, v, o, d, a, s);
 }
 
 }  // namespace
@@ -235,27 +265,16 @@ uint64_t calibatt_get_spin_limit_ns(void) { return spin_limit_ns(); }
 int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
                              int Np, int d, int dtype, float scale, const calibatt_blocklist* bl, int map_offset,
                              int32_t* dev_status, calibatt_stream_t stream) {
-  int rc = check_fwd(q, k, v, o, B, H, N, Np, d, dtype, scale, bl, map_offset);
-  if (rc) return rc;
-  const int nqb = Np / bl->block_q, nkb = Np / bl->block_k;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == CALIBATT_BF16) {
-    TcArgs a{};
-    a.B = B; a.H = H; a.N = N; a.Np = Np; a.nqb = nqb; a.nkb = nkb;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
-    a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
-    a.kscale = 128 / bl->block_k;
-    a.o = o; a.lse = lse; a.status = dev_status; a.spin_ns = spin_limit_ns();
-    return launch_tc_fwd(q, k, v, d, a, s);
-  }
-  SimtArgs a{};
-  a.B = B; a.H = H; a.N = N; a.Np = Np; a.block_q = bl->block_q; a.block_k = bl->block_k;
-  a.nqb = nqb; a.nkb = nkb; a.scale = scale;
-  a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
-  a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
-  a.lse = lse; a.status = dev_status;
-  return launch_simt_fwd(q, k, v, o, d, a, s);
+  return fwd_impl(q, k, v, o, lse, B, H, N, Np, N, Np, d, dtype, scale, bl, map_offset, dev_status, stream);
+}
+
+int calibatt_sparse_attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                int Nq, int Npq, int Nk, int Npk, int d, int dtype, float scale,
+                                const calibatt_blocklist* bl, int map_offset, int32_t* dev_status,
+                                calibatt_stream_t stream) {
+  if (dtype != CALIBATT_BF16)
+    return set_error(CALIBATT_E_UNSUPPORTED, "separate query and key lengths are supported for bf16 only");
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Npq, Nk, Npk, d, dtype, scale, bl, map_offset, dev_status, stream);
 }
 
 int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, const void* v_host, void* o_host,
@@ -270,7 +289,7 @@ int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, co
   if ((lse_host == nullptr) != (lse_dev == nullptr))
     return set_error(CALIBATT_E_INVALID, "lse_host and lse_dev must both be given or both be NULL");
   if (heads_per_chunk <= 0) return set_error(CALIBATT_E_INVALID, "heads_per_chunk must be >= 1");
-  int rc = check_fwd(q_dev, k_dev, v_dev, o_dev, B, H, N, Np, d, dtype, scale, bl, map_offset);
+  int rc = check_fwd(q_dev, k_dev, v_dev, o_dev, B, H, N, Np, N, Np, d, dtype, scale, bl, map_offset);
   if (rc) return rc;
   const size_t esize = dtype == CALIBATT_BF16 ? 2 : 4;
   const size_t plane = static_cast<size_t>(Np) * d * esize;   // bytes of one (b, h) slice

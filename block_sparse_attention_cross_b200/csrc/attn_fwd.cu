@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pol_q);
         ++qfills;
       }
-      const int row = score ? cs.bh * a.Np + cursor_kb(a, cs) * BK : cp.bh * a.Np + cursor_kb(a, cp) * BK;
+      const int row = score ? cs.bh * a.Npk + cursor_kb(a, cs) * BK : cp.bh * a.Npk + cursor_kb(a, cp) * BK;
       const int e = g % R;
       ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
       if (!ok) break;
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
-      const int valid_last = (kb_last == a.nkb - 1) ? (a.N - kb_last * BK) : BK;
+      const int valid_last = (kb_last == a.nkb - 1) ? (a.Nk - kb_last * BK) : BK;
       const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
       float m = -INFINITY;
       float l = 0.f;
@@ -662,12 +662,13 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 
 int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcArgs& a, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
-  const uint64_t rows = static_cast<uint64_t>(a.B) * a.H * a.Np;
+  const uint64_t qrows = static_cast<uint64_t>(a.B) * a.H * a.Np;
+  const uint64_t krows = static_cast<uint64_t>(a.B) * a.H * a.Npk;
   const uint32_t bk = static_cast<uint32_t>(TILE / a.kscale);   // key-block size: 128 or 64
   int rc;
-  if ((rc = make_tmap_bf16(&tq, q, rows, d, TILE)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tk, k, rows, d, bk)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tv, v, rows, d, bk)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tq, q, qrows, d, TILE)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, krows, d, bk)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, krows, d, bk)) != CALIBATT_OK) return rc;
   if (bk == 64) return d == 128 ? launch_fwd<128, 64>(tq, tk, tv, a, s) : launch_fwd<64, 64>(tq, tk, tv, a, s);
   return d == 128 ? launch_fwd<128, 128>(tq, tk, tv, a, s) : launch_fwd<64, 128>(tq, tk, tv, a, s);
 }

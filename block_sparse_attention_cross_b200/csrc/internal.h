@@ -18,7 +18,8 @@ uint64_t spin_limit_ns();
 
 // Kernel arguments of the tensor-core attention kernels.
 struct TcArgs {
-  int B, H, N, Np, nqb, nkb;
+  int B, H, N, Np, nqb, nkb;   // N, Np: query rows (real, padded)
+  int Nk, Npk;                 // forward: key rows (real, padded); equal to N, Np unless queries are gathered
   float scale_log2;
   const int32_t* row_base;
   const int32_t* row_pat;

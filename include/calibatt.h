@@ -177,6 +177,35 @@ int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, co
                                       int32_t* dev_status, calibatt_stream_t stream);
 
 /*
+ * calibatt_sparse_attn_fwd_qk -- the forward with different query and key
+ * lengths: Nq real query rows (padded to Npq) attend to Nk real keys (padded
+ * to Npk).  Used by the spatial-repetition path (paper page, Figure 5(b)
+ * bottom, Table S4), whose gathered anchor queries are fewer than the keys.
+ *  q, o  [B, H, Npq, d];  k, v  [B, H, Npk, d];  lse [B, H, Npq] or NULL.
+ *  bl    block list with block_q = 128, n_q_blocks = Npq / 128 and
+ *        n_k_blocks = Npk / block_k; Npq - Nq < 128, Npk - Nk < block_k.
+ * bf16 only (CALIBATT_E_UNSUPPORTED otherwise); other arguments, semantics and
+ * errors as calibatt_sparse_attn_fwd.
+ */
+int calibatt_sparse_attn_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                int Nq, int Npq, int Nk, int Npk, int d, int dtype, float scale,
+                                const calibatt_blocklist* bl, int map_offset, int32_t* dev_status,
+                                calibatt_stream_t stream);
+
+/*
+ * calibatt_gather_rows -- dst[p, i, :] = src[p, idx[i], :] for p < n_planes,
+ * i < rows_dst; an index outside [0, rows_src) writes a zero row.
+ * The spatial-repetition path (paper page, Figure 4 and Table S4) gathers the
+ * anchor query rows with it and broadcasts each anchor's output row to the
+ * rows it stands for.
+ *  src [n_planes, rows_src, row_bytes], dst [n_planes, rows_dst, row_bytes]
+ *  (device, 16-byte aligned, row_bytes a multiple of 16); idx [rows_dst]
+ *  int32 device.  Asynchronous.
+ */
+int calibatt_gather_rows(const void* src, void* dst, const int32_t* idx, int n_planes, int rows_src, int rows_dst,
+                         int row_bytes, calibatt_stream_t stream);
+
+/*
  * calibatt_block_energy -- block energies of one calibration input.
  *
  * Paper page, Figure 2 (block-level post-softmax attention maps) and

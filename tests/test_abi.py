@@ -183,3 +183,20 @@ def test_skiplist_validation(lib):
     assert lib.calibatt_interval_counts(fake, 0, 8, 8, fake, None) == _lib.E_INVALID
     assert lib.calibatt_merge_intervals(fake, 2, 8, 8, None, fake, None) == _lib.E_INVALID
     assert lib.calibatt_merge_intervals(fake, 2, 8, 4096, fake, fake, None) == _lib.E_UNSUPPORTED
+
+
+def test_gathered_query_forward_and_gather_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    bl = _blocklist(2, 2, 8, 128, 128)
+    # fp32 has no separate query / key lengths
+    assert lib.calibatt_sparse_attn_fwd_qk(fake, fake, fake, fake, None, 1, 2, 200, 256, 1000, 1024, 128, _lib.FP32,
+                                           0.1, ctypes.byref(bl), 0, None, None) == _lib.E_UNSUPPORTED
+    # query grid must match Npq / 128
+    assert lib.calibatt_sparse_attn_fwd_qk(fake, fake, fake, fake, None, 1, 2, 300, 384, 1000, 1024, 128, _lib.BF16,
+                                           0.1, ctypes.byref(bl), 0, None, None) == _lib.E_INVALID
+    # a whole padded query block is rejected
+    assert lib.calibatt_sparse_attn_fwd_qk(fake, fake, fake, fake, None, 1, 2, 100, 256, 1000, 1024, 128, _lib.BF16,
+                                           0.1, ctypes.byref(bl), 0, None, None) == _lib.E_INVALID
+    assert lib.calibatt_gather_rows(None, fake, fake, 1, 4, 4, 256, None) == _lib.E_INVALID
+    assert lib.calibatt_gather_rows(fake, fake, fake, 1, 4, 4, 200, None) == _lib.E_INVALID     # not a multiple of 16
+    assert lib.calibatt_gather_rows(ctypes.c_void_p(0x10008), fake, fake, 1, 4, 4, 256, None) == _lib.E_INVALID
