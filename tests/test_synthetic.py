@@ -77,3 +77,25 @@ def test_video_qkv_shapes_and_padding():
     # shared structure: Q and K of the same token are strongly correlated
     c = np.corrcoef(q[0, 0, :300].ravel(), k[0, 0, :300].ravel())[0, 1]
     assert c > 0.9
+
+
+def test_anchor_plan_indices_match_the_oracle_mapping():
+    # The host-side index lists of the spatial-repetition path: gathered query
+    # i is the token of anchor row a(i) of its frame, and every token's output
+    # comes from the gathered row of the token on its nearest anchor row.
+    import oracle
+    import block_sparse_attention_cross_b200 as cba
+    frames, rows, cols, k = 3, 7, 5, 3
+    N = frames * rows * cols
+    Np = (N + 127) // 128 * 128
+    plan = cba.anchor_plan(frames, rows, cols, k, Np, "cpu")
+    anchors, nearest = oracle.anchor_rows(rows, k)
+    assert (anchors, nearest) == cba.anchor_rows(rows, k)
+    iq = plan.idx_q.tolist()
+    io = plan.idx_o.tolist()
+    assert plan.nq == frames * k * cols and plan.npq % 128 == 0 and len(iq) == plan.npq
+    assert all(x == -1 for x in iq[plan.nq:]) and all(x == -1 for x in io[N:])
+    for t in range(N):
+        f, rem = divmod(t, rows * cols)
+        r, c = divmod(rem, cols)
+        assert iq[io[t]] == f * rows * cols + nearest[r] * cols + c
