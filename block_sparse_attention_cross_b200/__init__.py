@@ -30,7 +30,7 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
 __all__ = [
     "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
     "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "gather_rows",
-    "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "calibrate_schedule", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -480,6 +480,26 @@ def _nearest_rank(values, pct):
     v = torch.sort(values.reshape(-1).to(torch.int64)).values
     k = max(1, math.ceil(pct / 100.0 * v.numel()))
     return int(v[k - 1])
+
+
+def calibrate_schedule(inputs_per_step, N, param_of, select_mode=SELECT_ENERGY, rho=0.5, **kw):
+    """Calibration of every denoising step with its own selection parameter.
+
+    The paper page's energy threshold is a function of the normalized
+    timestep (Figure S8: epsilon against t/T; the values are not printed, so
+    the caller supplies them).  ``inputs_per_step``: for steps t = 0 .. T-1,
+    a pair (q_list, k_list) of that step's calibration inputs ([H, Np, d]
+    CUDA tensors); ``param_of(t, T)``: the selection parameter of step t
+    (epsilon for SELECT_ENERGY, the kept fraction for SELECT_TOPK).  Returns
+    uint8 masks [T, H, nqb, nkb], one :func:`calibrate` per step.
+    """
+    T = len(inputs_per_step)
+    masks = []
+    for t, (q_list, k_list) in enumerate(inputs_per_step):
+        m, _, _ = calibrate(q_list, k_list, N, select_mode=select_mode, select_param=float(param_of(t, T)), rho=rho,
+                            **kw)
+        masks.append(m)
+    return torch.stack(masks)
 
 
 def _compile_ws(n_maps, nqb, nkb, dev):

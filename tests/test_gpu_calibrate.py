@@ -169,3 +169,24 @@ def test_sharded_calibration_single_rank_matches_calibrate():
     assert torch.equal(votes1, votes2)
     assert torch.equal(esum1, esum2)
     assert torch.equal(mask1, mask2)
+
+
+def test_energy_schedule_per_timestep():
+    # One calibration per step with its own energy threshold (a schedule the
+    # caller supplies: the pages plot one but print no values); every step's
+    # mask equals the oracle's selection and vote on that step's GPU energies.
+    H = 2
+    steps = []
+    for t in range(3):
+        w, inputs = small_inputs(3, H, syn.VideoGrid(2, 20, 50), 128, seed_base=20 + t)
+        steps.append(([bf16_pair(q)[1] for q, _ in inputs], [bf16_pair(k)[1] for _, k in inputs]))
+    eps = lambda t, T: 0.05 + 0.3 * t / max(1, T - 1)
+    masks = cba.calibrate_schedule(steps, w.N, eps, rho=0.5)
+    assert masks.shape[0] == 3
+    for t, (qd, kd) in enumerate(steps):
+        Eg = [cba.block_energy(q, k, w.N).cpu().numpy() for q, k in zip(qd, kd)]
+        keeps = [oracle.select_energy(E, eps(t, 3)) for E in Eg]
+        m_o, _, _ = oracle.vote(np.stack(keeps), oracle.min_votes_for(0.5, 3), np.stack(Eg))
+        assert np.array_equal(masks[t].cpu().numpy(), m_o)
+    dens = [float(m.float().mean()) for m in masks]
+    print(f"PARITY energy schedule: 3 steps, densities {', '.join(f'{x:.3f}' for x in dens)}, masks bit-exact")
