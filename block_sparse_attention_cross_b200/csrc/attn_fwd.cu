@@ -44,6 +44,7 @@
 // completed).
 // Every wait is bounded; on expiry the CTA reports CALIBATT_E_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -621,38 +622,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-int g_num_sms = 0;
+std::atomic<int> g_num_sms{0};
 
 template <int D, int BK>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
                cudaStream_t s) {
   auto kern = k_attn_fwd<D, BK>;
   constexpr uint32_t smem_bytes = FwdLayout<D, BK>::SMEM_BYTES;
-  static bool configured = false;
-  if (!configured) {
+  // One-time set-up per instantiation; atomics keep concurrent first calls
+  // from several host threads race-free (the set-up itself is idempotent).
+  static std::atomic<bool> configured{false};
+  if (!configured.load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(k_attn_fwd)");
-    configured = true;
+    configured.store(true, std::memory_order_release);
   }
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
+  static std::atomic<int> launch_regs{-1};
+  int regs = launch_regs.load(std::memory_order_acquire);
+  if (regs < 0) {
     cudaFuncAttributes fa{};
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return check_launch("cudaFuncGetAttributes(k_attn_fwd)");
-    launch_regs = fa.numRegs;
+    regs = fa.numRegs;
+    launch_regs.store(regs, std::memory_order_release);
   }
   // The register re-split inside the kernel is sized for exactly kLaunchRegs
   // per thread at launch; refuse to launch a build with any other count.
-  if (launch_regs != kLaunchRegs)
-    return set_error(CALIBATT_E_UNSUPPORTED, "k_attn_fwd was built with %d registers per thread, expected %d",
-                     launch_regs, kLaunchRegs);
-  if (g_num_sms == 0) {
+  if (regs != kLaunchRegs)
+    return set_error(CALIBATT_E_UNSUPPORTED, "k_attn_fwd was built with %d registers per thread, expected %d", regs,
+                     kLaunchRegs);
+  int sms = g_num_sms.load(std::memory_order_acquire);
+  if (sms == 0) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return check_launch("cudaDeviceGetAttribute(SM count)");
+    g_num_sms.store(sms, std::memory_order_release);
   }
   const long long T = static_cast<long long>(a.B) * a.H * a.nqb;
-  const int grid = static_cast<int>(std::min<long long>(g_num_sms, T));
+  const int grid = static_cast<int>(std::min<long long>(sms, T));
   kern<<<grid, kThreads, smem_bytes, s>>>(tq, tk, tv, a);
   count_launch();
   return check_launch("k_attn_fwd");

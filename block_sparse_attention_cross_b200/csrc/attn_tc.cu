@@ -19,6 +19,7 @@
 // elected lane.  Every wait is bounded; on expiry the CTA records
 // CALIBATT_E_TIMEOUT, waits (bounded) for its own copies and MMAs, frees TMEM
 // and exits.
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -248,12 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int MODE>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const TcArgs& a, dim3 grid, cudaStream_t s) {
   auto kern = k_energy_tc<D, MODE>;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<bool> configured{false};   // one-time, idempotent set-up; race-free across host threads
+  if (!configured.load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, EnergyLayout<D>::SMEM_BYTES) !=
         cudaSuccess)
       return check_launch("cudaFuncSetAttribute(k_energy_tc)");
-    configured = true;
+    configured.store(true, std::memory_order_release);
   }
   kern<<<grid, kThreads, EnergyLayout<D>::SMEM_BYTES, s>>>(tq, tk, a);
   count_launch();
