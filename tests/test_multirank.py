@@ -95,3 +95,14 @@ def test_sharded_calibration_gathers_inputs_in_global_order_gloo(world):
     for rank in range(world):
         assert out[rank][:-1] == [float(i) for i in range(n)]
         assert out[rank][-1] == (2, 3, 4)
+
+
+def test_bench_workload_helpers():
+    # FLOPs per kept block follow the block shape; the _k64 workload is the
+    # 480p call with 64-key blocks.
+    assert bench.kept_flops(1, 128, 1) == 4.0 * 128 * 128 * 128
+    assert bench.kept_flops(2, 128, 1, block_k=64) == bench.kept_flops(1, 128, 1)
+    assert bench.key_block("wan480_25_k64") == 64 and bench.key_block("wan480_25") == 128
+    w = bench.workload(None, "wan480_25_k64")
+    assert (w.name, w.N, w.H) == ("wan480_25", 32760, 40)
+    assert bench.workload(8, "sweep").H == 8
