@@ -41,7 +41,12 @@
 // halves exchange their block maxima after their stores are in flight.  Only
 // when a row's block max exceeds m by more than kRescaleThreshold is the
 // block redone with the raised m and O rescaled (after the previous PV has
-// completed).
+// completed).  Each tile walks its list from the first kept block at or after
+// its own (diagonal) block, wrapping around, so the first block usually holds
+// the row max.  The epilogue moves the bf16 rounding error of each half's
+// largest probability into the normaliser (see the epilogue).
+// Query rows (N, Np) and key rows (Nk, Npk) may differ: gathered anchor
+// queries attend to the whole sequence.
 // Every wait is bounded; on expiry the CTA reports CALIBATT_E_TIMEOUT, drains
 // its own copies and MMAs, frees TMEM and exits.
 #include <atomic>
