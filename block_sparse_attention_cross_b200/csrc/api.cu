@@ -55,6 +55,14 @@ uint64_t spin_limit_ns() {
   return g_spin_ns.load();
 }
 
+int current_device(int* dev) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return check_launch("cudaGetDevice");
+  if (d < 0 || d >= kMaxDevices) return set_error(CALIBATT_E_UNSUPPORTED, "device ordinal %d out of range", d);
+  *dev = d;
+  return CALIBATT_OK;
+}
+
 // ---- TMA descriptors --------------------------------------------------------
 
 namespace {
@@ -219,11 +227,11 @@ struct StreamSet {
   cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
 };
 std::mutex g_stream_mu;
-StreamSet g_streams[64];
+StreamSet g_streams[kMaxDevices];
 
 int stream_set(StreamSet** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return check_launch("cudaGetDevice");
+  if (int rc = current_device(&dev)) return rc;
   StreamSet& ss = g_streams[dev];
   if (ss.h2d == nullptr) {
     if (cudaStreamCreateWithFlags(&ss.h2d, cudaStreamNonBlocking) != cudaSuccess ||
@@ -353,7 +361,9 @@ int calibatt_calibrate_workspace_size(int H, int N, int Np, int d, int block_q, 
   return CALIBATT_OK;
 }
 
-namespace {
+}  // extern "C"
+
+namespace calibatt {
 
 int energy_impl(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int block_q, int block_k,
                 float scale, float* energy_out, float* lse_ws, int32_t* dev_status, cudaStream_t s) {
@@ -394,6 +404,12 @@ int check_energy_args(const void* q, const void* k, int H, int N, int Np, int d,
   }
   return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
 }
+
+}  // namespace calibatt
+
+extern "C" {
+
+namespace {
 
 int carve_energy_ws(void* ws, size_t ws_bytes, int H, int N, int Np, int d, int bq, int bk, float** lse,
                     float** energy) {

@@ -71,12 +71,6 @@ constexpr uint32_t kTmemCols = 512;
 // exceeds it by more than this many log2 units, so every P <= 2^64; row sums
 // and O stay far below the fp32 range for |v| < 2^47.
 constexpr float kRescaleThreshold = 64.0f;
-// Column pairs i with (i % 8) >= kPolyFrom evaluate exp2 with the FMA-pipe
-// polynomial instead of MUFU.  Measured on B200 at this instruction mix the
-// MUFU unit is not the limiter, so the polynomial is off (8).  The epilogue's
-// normaliser fix-up re-forms one probability with MUFU, so it is exact only
-// while the polynomial is off.
-constexpr int kPolyFrom = 8;
 
 // D: head dim; BK: key-block size (128 or 64; query blocks are always 128).
 template <int D, int BK>
@@ -459,8 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < HB; ++i)
             if (h * HB + i >= valid_last) r[i] = f2u(-INFINITY);
         }
-        // p = 2^(s c2 - mref) two columns at a time (pairs selected by
-        // kPolyFrom use the FMA-pipe polynomial, the rest the MUFU unit), as
+        // p = 2^(s c2 - mref) two columns at a time on the MUFU unit, as
         // bf16 pairs into the first 32 columns of this half's score columns,
         // 16 columns (32 probabilities) per store.  Returns the half-row sum;
         // with `track` it also returns the half-row maximum of the raw scores.
@@ -480,14 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else mxa = fmax3(mxa, u2f(r[e]), u2f(r[e + 1]));
               }
               const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
-              uint64_t pv;
-              if ((i & 7) >= kPolyFrom) {
-                pv = exp2_poly2(x);
-              } else {
-                float xl, xh;
-                f2unpack(x, xl, xh);
-                pv = f2pack(ex2_approx(xl), ex2_approx(xh));
-              }
+              float xl, xh;
+              f2unpack(x, xl, xh);
+              const uint64_t pv = f2pack(ex2_approx(xl), ex2_approx(xh));
               if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
               float pl, ph;
               f2unpack(pv, pl, ph);
@@ -627,20 +615,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
-std::atomic<int> g_num_sms{0};
+// SM count of every device, looked up on its first launch there.
+std::atomic<int> g_num_sms[kMaxDevices];
 
 template <int D, int BK>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
                cudaStream_t s) {
   auto kern = k_attn_fwd<D, BK>;
   constexpr uint32_t smem_bytes = FwdLayout<D, BK>::SMEM_BYTES;
-  // One-time set-up per instantiation; atomics keep concurrent first calls
+  int dev = 0;
+  if (int rc = current_device(&dev)) return rc;
+  // One-time set-up per instantiation and device (the shared-memory limit is
+  // a per-device function attribute); atomics keep concurrent first calls
   // from several host threads race-free (the set-up itself is idempotent).
-  static std::atomic<bool> configured{false};
-  if (!configured.load(std::memory_order_acquire)) {
+  static std::atomic<bool> configured[kMaxDevices];
+  if (!configured[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(k_attn_fwd)");
-    configured.store(true, std::memory_order_release);
+    configured[dev].store(true, std::memory_order_release);
   }
   static std::atomic<int> launch_regs{-1};
   int regs = launch_regs.load(std::memory_order_acquire);
@@ -655,13 +647,11 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
   if (regs != kLaunchRegs)
     return set_error(CALIBATT_E_UNSUPPORTED, "k_attn_fwd was built with %d registers per thread, expected %d", regs,
                      kLaunchRegs);
-  int sms = g_num_sms.load(std::memory_order_acquire);
+  int sms = g_num_sms[dev].load(std::memory_order_acquire);
   if (sms == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return check_launch("cudaDeviceGetAttribute(SM count)");
-    g_num_sms.store(sms, std::memory_order_release);
+    g_num_sms[dev].store(sms, std::memory_order_release);
   }
   const long long T = static_cast<long long>(a.B) * a.H * a.nqb;
   const int grid = static_cast<int>(std::min<long long>(sms, T));

@@ -249,12 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int MODE>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const TcArgs& a, dim3 grid, cudaStream_t s) {
   auto kern = k_energy_tc<D, MODE>;
-  static std::atomic<bool> configured{false};   // one-time, idempotent set-up; race-free across host threads
-  if (!configured.load(std::memory_order_acquire)) {
+  int dev = 0;
+  if (int rc = current_device(&dev)) return rc;
+  // One-time, idempotent set-up per device (the shared-memory limit is a
+  // per-device function attribute); race-free across host threads.
+  static std::atomic<bool> configured[kMaxDevices];
+  if (!configured[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, EnergyLayout<D>::SMEM_BYTES) !=
         cudaSuccess)
       return check_launch("cudaFuncSetAttribute(k_energy_tc)");
-    configured.store(true, std::memory_order_release);
+    configured[dev].store(true, std::memory_order_release);
   }
   kern<<<grid, kThreads, EnergyLayout<D>::SMEM_BYTES, s>>>(tq, tk, a);
   count_launch();

@@ -441,35 +441,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two lanes on the FMA pipe instead of the MUFU unit.  Method:
-// round-to-nearest range reduction x = n + f, f in [-1/2, 1/2] (adding
-// 1.5 * 2^23 leaves n in the low mantissa bits), a degree-3 polynomial for
-// 2^f fitted here for minimum relative error on [-1/2, 1/2] (max relative
-// error 1.0e-4, below the bf16 rounding applied to probabilities), and
-// n added to the exponent field.  Inputs are clamped to >= -126 so the
-// exponent cannot wrap; results below 2^-126 are negligible here.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
-  float xl, xh;
-  f2unpack(x, xl, xh);
-  x = f2pack(fmaxf(xl, -126.f), fmaxf(xh, -126.f));
-  const uint64_t kMagic = f2pack(12582912.f, 12582912.f);
-  const uint64_t kNegMagic = f2pack(-12582912.f, -12582912.f);
-  const uint64_t kNegOne = f2pack(-1.f, -1.f);
-  const uint64_t t = fadd2(x, kMagic);
-  const uint64_t n = fadd2(t, kNegMagic);
-  const uint64_t f = ffma2(n, kNegOne, x);
-  uint64_t p = ffma2(f2pack(0.05500892922282219f, 0.05500892922282219f), f,
-                     f2pack(0.24221095442771912f, 0.24221095442771912f));
-  p = ffma2(p, f, f2pack(0.6932829022407532f, 0.6932829022407532f));
-  p = ffma2(p, f, f2pack(1.f, 1.f));
-  float tl, th, pl, ph;
-  f2unpack(t, tl, th);
-  f2unpack(p, pl, ph);
-  const uint32_t rl = __float_as_uint(pl) + (__float_as_uint(tl) << 23);
-  const uint32_t rh = __float_as_uint(ph) + (__float_as_uint(th) << 23);
-  return f2pack(__uint_as_float(rl), __uint_as_float(rh));
-}
-
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 }  // namespace calibatt

@@ -16,6 +16,12 @@ int check_launch(const char* what);   // cudaGetLastError -> status
 void count_launch(int n = 1);
 uint64_t spin_limit_ns();
 
+// One-time launch set-up (dynamic shared-memory limits, SM counts, symbol
+// addresses) is a per-device property: it is kept per device ordinal.
+constexpr int kMaxDevices = 64;
+// The current device's ordinal, checked against kMaxDevices.
+int current_device(int* dev);
+
 // Kernel arguments of the tensor-core attention kernels.
 struct TcArgs {
   int B, H, N, Np, nqb, nkb;   // N, Np: query rows (real, padded)
@@ -47,6 +53,14 @@ struct SimtArgs {
   float* energy;     // calibration: [H, nqb, nkb]
   int32_t* status;
 };
+
+// Argument checks and launch of the block energies, shared by
+// calibatt_block_energy, calibatt_calibrate and calibatt_block_energy_noalloc
+// (api.cu).  lse_ws: per-row scratch of H * Np floats.
+int check_energy_args(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int block_q,
+                      int block_k, float scale);
+int energy_impl(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int block_q, int block_k,
+                float scale, float* energy_out, float* lse_ws, int32_t* dev_status, cudaStream_t s);
 
 // attn_tc.cu (bf16, tcgen05)
 int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcArgs& a, cudaStream_t s);

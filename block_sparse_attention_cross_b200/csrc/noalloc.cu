@@ -15,7 +15,6 @@
 // streams, or different host threads on the same device) race on it; calls
 // on one stream are ordered and safe.  The first pass of every call writes
 // each scratch entry it later reads, so nothing needs clearing between calls.
-#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -25,7 +24,6 @@ namespace calibatt {
 namespace {
 
 constexpr long long kNoallocScratchFloats = 4ll * 1024 * 1024;  // 16 MiB: H * Np <= 4 Mi rows
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchFloats];
 
@@ -37,8 +35,7 @@ float* g_noalloc_ptr[kMaxDevices] = {};
 // address is looked up once per device, with that device current.
 int scratch_for_current_device(float** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return set_error(CALIBATT_E_UNSUPPORTED, "device ordinal %d out of range", dev);
+  if (int rc = current_device(&dev)) return rc;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (g_noalloc_ptr[dev] == nullptr) {
     void* p = nullptr;
@@ -58,47 +55,21 @@ int scratch_for_current_device(float** out) {
 
 using namespace calibatt;
 
+// Same validation and launch path as calibatt_block_energy; only the source
+// of the per-row scratch differs.
 extern "C" int calibatt_block_energy_noalloc(const void* q, const void* k, int H, int N, int Np, int d, int dtype,
                                              int block_q, int block_k, float scale, float* energy_out,
                                              int32_t* dev_status, calibatt_stream_t stream) {
-  if (q == nullptr || k == nullptr || energy_out == nullptr)
-    return set_error(CALIBATT_E_INVALID, "q, k and energy_out must be non-NULL");
-  if (H <= 0 || N <= 0 || Np < N || d <= 0 || block_q <= 0 || block_k <= 0 || Np % block_q || Np % block_k)
-    return set_error(CALIBATT_E_INVALID, "bad sizes H=%d N=%d Np=%d d=%d", H, N, Np, d);
-  if ((Np - N) >= block_k || (Np - N) >= block_q)
-    return set_error(CALIBATT_E_INVALID, "Np - N must be smaller than one block");
-  if (!(scale > 0.f) || !std::isfinite(scale)) return set_error(CALIBATT_E_INVALID, "scale must be finite and > 0");
-  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) & 15u)
-    return set_error(CALIBATT_E_INVALID, "q and k must be 16-byte aligned");
+  int rc = check_energy_args(q, k, H, N, Np, d, dtype, block_q, block_k, scale);
+  if (rc) return rc;
+  if (energy_out == nullptr) return set_error(CALIBATT_E_INVALID, "energy_out is NULL");
   if (static_cast<long long>(H) * Np > kNoallocScratchFloats)
     return set_error(CALIBATT_E_WORKSPACE,
                      "H * Np = %lld rows exceeds the built-in scratch of %lld rows; use calibatt_block_energy "
                      "with a workspace",
                      static_cast<long long>(H) * Np, kNoallocScratchFloats);
-  const int nqb = Np / block_q, nkb = Np / block_k;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == CALIBATT_BF16) {
-    if (!(d == 64 || d == 128) || block_q != 128 || block_k != 128)
-      return set_error(CALIBATT_E_UNSUPPORTED, "bf16 energies support d in {64,128} with 128x128 blocks");
-    if (nkb > 1024) return set_error(CALIBATT_E_UNSUPPORTED, "at most 1024 key blocks");
-  } else if (dtype == CALIBATT_FP32) {
-    if (!(d == 64 || d == 128) || !(block_q == 64 || block_q == 128) || !(block_k == 64 || block_k == 128))
-      return set_error(CALIBATT_E_UNSUPPORTED, "fp32 energies support d in {64,128}, blocks in {64,128}");
-  } else {
-    return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
-  }
   float* scratch = nullptr;
-  int rc = scratch_for_current_device(&scratch);
-  if (rc) return rc;
-  if (dtype == CALIBATT_BF16) {
-    TcArgs a{};
-    a.B = 1; a.H = H; a.N = N; a.Np = Np; a.nqb = nqb; a.nkb = nkb;
-    a.scale_log2 = scale * 1.4426950408889634f;
-    a.lse2 = scratch; a.energy = energy_out; a.status = dev_status; a.spin_ns = spin_limit_ns();
-    return launch_tc_energy(q, k, d, a, s);
-  }
-  SimtArgs a{};
-  a.B = 1; a.H = H; a.N = N; a.Np = Np; a.block_q = block_q; a.block_k = block_k; a.nqb = nqb; a.nkb = nkb;
-  a.scale = scale; a.lse = scratch; a.energy = energy_out; a.status = dev_status;
-  return launch_simt_energy(q, k, d, a, s);
+  if ((rc = scratch_for_current_device(&scratch))) return rc;
+  return energy_impl(q, k, H, N, Np, d, dtype, block_q, block_k, scale, energy_out, scratch, dev_status,
+                     reinterpret_cast<cudaStream_t>(stream));
 }

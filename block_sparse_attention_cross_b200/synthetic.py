@@ -15,18 +15,22 @@ their attention shapes.
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
+
+
+def _threads():
+    return max(1, min(16, len(os.sched_getaffinity(0))))
 
 # --------------------------------------------------------------------------
 # bf16 helpers (round-to-nearest-even on the float32 bit pattern)
 # --------------------------------------------------------------------------
 
 
-def f32_to_bf16_bits(x):
-    """Round float32 values to bf16 (nearest even); returns uint16 bit patterns."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
+def _bf16_bits_chunk(x):
     u = x.view(np.uint32).astype(np.uint64)
     rounding = ((u >> 16) & 1) + 0x7FFF
     out = ((u + rounding) >> 16).astype(np.uint16)
@@ -34,6 +38,28 @@ def f32_to_bf16_bits(x):
     if nan.any():
         out[nan] = 0x7FC0
     return out
+
+
+def f32_to_bf16_bits(x):
+    """Round float32 values to bf16 (nearest even); returns uint16 bit patterns.
+
+    Large arrays are rounded in chunks on a thread pool (numpy releases the
+    GIL); the result does not depend on the chunking.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    flat = x.reshape(-1)
+    if flat.size < (1 << 22):
+        return _bf16_bits_chunk(flat).reshape(x.shape)
+    out = np.empty(flat.size, dtype=np.uint16)
+    step = 1 << 21
+    starts = range(0, flat.size, step)
+
+    def work(i):
+        out[i:i + step] = _bf16_bits_chunk(flat[i:i + step])
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(work, starts))
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(bits):
@@ -156,9 +182,13 @@ def video_qk_base(grid: VideoGrid, H, d, seed, rank=16, alpha=1.0, jitter=0.0, j
         X = X + jitter * jr.standard_normal(X.shape)
     f, y, x = _token_coords(grid)
     base = np.empty((H, grid.video_tokens, d), dtype=np.float32)
-    for h in range(H):
+
+    def head(h):
         lat = F[h][f] + Y[h][y] + X[h][x]
         base[h] = (alpha * (lat @ W[h])).astype(np.float32)
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(head, range(H)))
     return base
 
 
@@ -168,33 +198,39 @@ def video_qkv(w: Workload, noise=0.1, with_v=True, input_index=None, jitter=0.05
     Q and K share the low-rank base and get independent N(0, noise^2) noise;
     text tokens (if any) and V are N(0, 1); padding rows are 0.  With
     ``input_index`` = n the base gets a per-input jitter and the noise comes
-    from seed 100 + n (calibration inputs).
+    from seeds derived from 100 + n (calibration inputs).  Every (tensor,
+    batch, head) slice draws from its own stream, seeded by (seed, b, h), so
+    the slices are filled in parallel and the values do not depend on the
+    thread count.
     """
     g = w.grid
     s = w.seeds
     if input_index is None:
         base = video_qk_base(g, w.H, w.d, s["base"])
-        rq = np.random.default_rng(s["noise_q"])
-        rk = np.random.default_rng(s["noise_k"])
+        sq, sk = [s["noise_q"]], [s["noise_k"]]
     else:
         base = video_qk_base(g, w.H, w.d, s["base"], jitter=jitter, jitter_seed=100 + input_index)
-        rq = np.random.default_rng([100 + input_index, 1])
-        rk = np.random.default_rng([100 + input_index, 2])
+        sq, sk = [100 + input_index, 1], [100 + input_index, 2]
+    sv = [s.get("v", 0)]
     Nv, N, Np = g.video_tokens, w.N, w.Np
     q = np.zeros((w.B, w.H, Np, w.d), dtype=np.float32)
     k = np.zeros_like(q)
-    for b in range(w.B):
-        for h in range(w.H):
-            q[b, h, :Nv] = base[h] + noise * rq.standard_normal((Nv, w.d), dtype=np.float32)
-            k[b, h, :Nv] = base[h] + noise * rk.standard_normal((Nv, w.d), dtype=np.float32)
+    v = np.zeros_like(q) if with_v else None
+
+    def plane(bh):
+        b, h = divmod(bh, w.H)
+        for x, seed in ((q, sq), (k, sk)):
+            r = np.random.default_rng(seed + [b, h])
+            x[b, h, :Nv] = base[h] + noise * r.standard_normal((Nv, w.d), dtype=np.float32)
             if N > Nv:
-                q[b, h, Nv:N] = rq.standard_normal((N - Nv, w.d), dtype=np.float32)
-                k[b, h, Nv:N] = rk.standard_normal((N - Nv, w.d), dtype=np.float32)
+                x[b, h, Nv:N] = r.standard_normal((N - Nv, w.d), dtype=np.float32)
+        if v is not None:
+            v[b, h, :N] = np.random.default_rng(sv + [b, h]).standard_normal((N, w.d), dtype=np.float32)
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(plane, range(w.B * w.H)))
     if not with_v:
         return q, k
-    rv = np.random.default_rng(s.get("v", 0))
-    v = np.zeros_like(q)
-    v[:, :, :N] = rv.standard_normal((w.B, w.H, N, w.d), dtype=np.float32)
     return q, k, v
 
 

@@ -43,7 +43,7 @@ pages print no epsilon values, so its *schedule* is unpinned (parity unpinned
 for epsilon values, not for the selection rule).
 """
 
-from .attention import masked_attention, masked_attention_rows, dense_attention_lse
+from .attention import masked_attention, masked_attention_rows
 from .calibration import block_energy, select_topk, select_energy, topk_count, vote, min_votes_for
 from .compile import compile_blocklist, expand_blocklist
 from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
@@ -53,7 +53,6 @@ from .anchor import anchor_rows, anchor_attention
 __all__ = [
     "masked_attention",
     "masked_attention_rows",
-    "dense_attention_lse",
     "block_energy",
     "select_topk",
     "select_energy",

@@ -100,14 +100,3 @@ def masked_attention(q, k, v, mask, N, block_q, block_k, scale):
                 LSE[b, h, qb * block_q:(qb + 1) * block_q] = lse
     return O, LSE
 
-
-def dense_attention_lse(q_h, k_h, N, scale):
-    """Row log-sum-exp of dense (unmasked) attention for one head: rows < N.
-
-    Used by the block-energy definition; returns LSE [N] in float64.
-    """
-    q_h = _as_f64(q_h)[:N]
-    k_h = _as_f64(k_h)[:N]
-    s = float(np.float64(scale)) * (q_h @ k_h.T)
-    m = s.max(axis=1)
-    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
