@@ -44,11 +44,11 @@ for epsilon values, not for the selection rule).
 """
 
 from .attention import masked_attention, masked_attention_rows
-from .calibration import block_energy, select_topk, select_energy, topk_count, vote, min_votes_for
+from .calibration import block_energy, block_energy_row, select_topk, select_energy, topk_count, vote, min_votes_for
 from .compile import compile_blocklist, expand_blocklist
 from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
 from .skiplist import interval_counts, merge_row, merge_masks, nearest_rank, skiplist_bytes
-from .anchor import anchor_rows, anchor_attention
+from .anchor import anchor_rows, anchor_attention, anchor_attention_tokens
 
 __all__ = [
     "masked_attention",

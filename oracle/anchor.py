@@ -57,3 +57,26 @@ def anchor_attention(q, k, v, N, frames, rows, cols, k_anchor, scale):
                     cache[ta] = (p @ v[b, h, :N]) / p.sum()
                 out[b, h, t] = cache[ta]
     return out
+
+
+def anchor_attention_tokens(q, k, v, N, frames, rows, cols, k_anchor, scale, b, h, tokens):
+    """O8 for selected tokens of (batch b, head h): [len(tokens), d] float64.
+
+    Token t takes softmax(scale q_a K^T) V of its anchor token a (same frame
+    and column, nearest anchor row) over the real keys; for full-size inputs,
+    where computing every token is too slow.
+    """
+    kh = np.asarray(k[b, h, :N], np.float64)
+    vh = np.asarray(v[b, h, :N], np.float64)
+    _, nearest = anchor_rows(rows, k_anchor)
+    out = np.zeros((len(tokens), vh.shape[1]))
+    for i, t in enumerate(tokens):
+        if t >= N:
+            continue
+        f, rem = divmod(int(t), rows * cols)
+        r, c = divmod(rem, cols)
+        ta = f * rows * cols + nearest[r] * cols + c
+        s = scale * (kh @ np.asarray(q[b, h, ta], np.float64))
+        p = np.exp(s - s.max())
+        out[i] = (p @ vh) / p.sum()
+    return out

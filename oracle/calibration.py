@@ -34,6 +34,21 @@ import math
 import numpy as np
 
 
+def _energy_row(q_rows, k_real, N, block_k, nkb, scale):
+    """E[qb, :] of one query block: its real rows ``q_rows`` against the real keys."""
+    s = scale * (q_rows @ k_real.T)              # [rows, N] dense scores
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    p /= p.sum(axis=1, keepdims=True)            # dense softmax rows
+    col_mass = p.sum(axis=0)                     # summed over the block's rows
+    row = np.zeros(nkb)
+    for kb in range(nkb):
+        c0, c1 = kb * block_k, min((kb + 1) * block_k, N)
+        if c1 > c0:
+            row[kb] = col_mass[c0:c1].sum() / q_rows.shape[0]
+    return row
+
+
 def block_energy(q, k, N, block_q, block_k, scale):
     """Block energies of one calibration input.
 
@@ -54,16 +69,20 @@ def block_energy(q, k, N, block_q, block_k, scale):
             r1 = min(r0 + block_q, N)
             if r1 <= r0:
                 continue
-            s = scale * (q[h, r0:r1] @ kh.T)          # [rows, N] dense scores
-            m = s.max(axis=1, keepdims=True)
-            p = np.exp(s - m)
-            p /= p.sum(axis=1, keepdims=True)        # dense softmax rows
-            col_mass = p.sum(axis=0)                 # summed over the block's rows
-            for kb in range(nkb):
-                c0, c1 = kb * block_k, min((kb + 1) * block_k, N)
-                if c1 > c0:
-                    E[h, qb, kb] = col_mass[c0:c1].sum() / (r1 - r0)
+            E[h, qb] = _energy_row(q[h, r0:r1], kh, N, block_k, nkb, scale)
     return E
+
+
+def block_energy_row(q, k, N, block_q, block_k, scale, h, qb):
+    """One row E[h, qb, :] of ``block_energy`` (for sampled checks at full size)."""
+    Np = np.shape(q)[1]
+    nkb = Np // block_k
+    r0, r1 = qb * block_q, min(qb * block_q + block_q, N)
+    if r1 <= r0:
+        return np.zeros(nkb)
+    qh = np.asarray(q[h, r0:r1], dtype=np.float64)
+    kh = np.asarray(k[h, :N], dtype=np.float64)
+    return _energy_row(qh, kh, N, block_k, nkb, float(np.float64(scale)))
 
 
 def topk_count(frac, nkb):

@@ -112,6 +112,47 @@ def test_calibrate_small_end_to_end():
 
 
 @pytest.mark.slow
+def test_calibrate_wan_config_full_size_against_float64_oracle():
+    # The calibration workload at full size: 8 Wan 480p inputs (40 heads,
+    # 32 760 tokens).  For 4 heads the float64 oracle scores every input: the
+    # GPU's energies must match element by element, and the masks that the
+    # oracle's selection and vote build from its own float64 energies may
+    # differ from the GPU's masks only in near-tie rows.
+    from _oracle_pool import block_energies
+    w = syn.WORKLOADS["wan480_25"]
+    I, heads = 8, [0, 13, 26, 39]
+    scale = cba.default_scale(w.d)
+    qd, kd, jobs = [], [], []
+    for n in range(I):
+        q, k = syn.video_qkv(w, with_v=False, input_index=n)
+        q64, qg = bf16_pair(q[0])
+        k64, kg = bf16_pair(k[0])
+        qd.append(qg)
+        kd.append(kg)
+        jobs += [(q64[h:h + 1].copy(), k64[h:h + 1].copy(), w.N, 128, scale) for h in heads]
+        del q, k, q64, k64
+    mask, votes, esum = cba.calibrate(qd, kd, w.N, select_param=0.25, rho=0.5)
+    Eg = np.stack([cba.block_energy(q, k, w.N)[heads].cpu().numpy() for q, k in zip(qd, kd)])
+    mask_g = mask[heads].cpu().numpy()
+    del qd, kd
+    torch.cuda.empty_cache()
+    Eo = np.stack(block_energies(jobs)).reshape(I, len(heads), w.nqb, w.nqb)
+    err = np.abs(Eg.astype(np.float64) - Eo)
+    print(f"PARITY energy wan480 8 inputs x {len(heads)} heads: max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
+    assert err.max() <= 5e-5
+    k = oracle.topk_count(0.25, w.nqb)
+    keeps = [oracle.select_topk(E, 0.25) for E in Eo]
+    m64, _, _ = oracle.vote(np.stack(keeps), oracle.min_votes_for(0.5, I), Eo)
+    tie = np.zeros((len(heads), w.nqb), bool)
+    for E in Eo:
+        tie |= near_tie_rows(E, k)
+    diff_rows = (mask_g != m64).any(axis=-1)
+    print(f"PARITY calibrate wan480 end to end: rows_differing={int(diff_rows.sum())} "
+          f"near_tie_rows={int(tie.sum())} of {tie.size}")
+    assert not (diff_rows & ~tie).any()
+
+
+@pytest.mark.slow
 def test_calibrate_wan_config_subset():
     # 8 calibration inputs of the Wan 480p shape; the oracle's discrete stages
     # run on the GPU's energies for every head.

@@ -106,3 +106,50 @@ def test_bench_workload_helpers():
     w = bench.workload(None, "wan480_25_k64")
     assert (w.name, w.N, w.H) == ("wan480_25", 32760, 40)
     assert bench.workload(8, "sweep").H == 8
+
+
+def _replica_probe(path):
+    # one replica of the harness on CPU: the torchrun-style environment set by
+    # launch_replicas, a gloo group, the max-over-ranks timing and the line
+    import json
+    world, rank, local = bench.dist_env()
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t_max = bench.max_over_ranks([100.0, 125.0][rank], dist, torch.device("cpu"))
+        line = bench.contract_line(world, 10, 3, t_max, 5.0e12, {"workload": "probe"})
+        with open(f"{path}.{rank}", "w") as f:
+            f.write(json.dumps({"line": line, "local": local, "addr": os.environ["MASTER_ADDR"]}))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gpus_2_launches_two_replica_ranks_gloo(tmp_path):
+    import json
+    codes = bench.launch_replicas(2, _replica_probe, (str(tmp_path / "out"),))
+    assert codes == [0, 0]
+    for rank in range(2):
+        rec = json.loads((tmp_path / f"out.{rank}").read_text())
+        line = rec["line"]
+        assert rec["local"] == rank and rec["addr"] == "127.0.0.1"
+        assert line["n_gpus"] == 2 and line["scaling"] == "weak" and line["steps"] == 10
+        assert line["ms_per_step"] == 12.5                         # the slower rank's 125 ms over 10 steps
+        assert line["value"] == pytest.approx(2 * 5.0e12 * 10 / 0.125 / 1e12, rel=1e-3)
+        assert line["config"]["parallelism"].startswith("replicas x2")
+
+
+def test_main_spawns_replicas_without_a_launcher(monkeypatch):
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench, "launch_replicas", lambda n, target, args=(): calls.append((n, target, args)) or [0] * n)
+    monkeypatch.setattr(bench.sys, "argv", ["bench.py", "--gpus", "2", "--steps", "4"])
+    bench.main()
+    assert calls and calls[0][0] == 2 and calls[0][1] is bench._replica_main
+    assert calls[0][2] == (["--gpus", "2", "--steps", "4"],)
+
+
+def test_main_refuses_a_world_size_other_than_gpus(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(bench.sys, "argv", ["bench.py", "--gpus", "4"])
+    with pytest.raises(SystemExit, match="WORLD_SIZE=2"):
+        bench.main()

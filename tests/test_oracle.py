@@ -503,3 +503,20 @@ def test_anchor_attention_against_sdpa():
                 t = f * rows * cols + r * cols + c
                 ta = f * rows * cols + nearest[r] * cols + c
                 assert np.allclose(o[:, :, t], ref[:, :, ta], atol=1e-12)
+    # the per-token form: the same values for a token subset, zeros past N
+    toks = [0, 7, 31, N - 1, N + 2]
+    for h in range(2):
+        sub = oracle.anchor_attention_tokens(q, k, v, N, frames, rows, cols, 2, scale, 0, h, toks)
+        want = [ref[0, h, f * rows * cols + nearest[(t % (rows * cols)) // cols] * cols + t % cols]
+                if t < N else np.zeros(d) for t in toks for f in [t // (rows * cols)]]
+        assert np.allclose(sub, np.stack(want), atol=1e-12)
+
+
+def test_block_energy_row_is_a_row_of_block_energy():
+    rng = np.random.default_rng(5)
+    H, N, Np, d = 2, 300, 384, 16
+    q = rng.standard_normal((H, Np, d))
+    k = rng.standard_normal((H, Np, d))
+    E = oracle.block_energy(q, k, N, 128, 64, 0.25)
+    for h, qb in ((0, 0), (1, 2), (1, 1)):
+        assert np.array_equal(oracle.block_energy_row(q, k, N, 128, 64, 0.25, h, qb), E[h, qb])
