@@ -217,10 +217,12 @@ def gather_rows(src, idx, rows_dst=None):
 def anchor_rows(rows, k):
     """The k anchor rows of a frame of ``rows`` spatial rows, evenly spaced and
     centred, and for every row the anchor it takes its output from (the
-    nearest, the lower one on a tie)."""
-    anchors = [int(math.floor((i + 0.5) * rows / k)) for i in range(k)]
-    nearest = [min(anchors, key=lambda a: (abs(a - r), a)) for r in range(rows)]
-    return anchors, nearest
+    nearest, the lower one on a tie): ``calibatt_anchor_rows``."""
+    anchors = np.zeros(int(k), dtype=np.int32)
+    nearest = np.zeros(int(rows), dtype=np.int32)
+    check(load().calibatt_anchor_rows(int(rows), int(k), anchors.ctypes.data_as(ctypes.c_void_p),
+                                      nearest.ctypes.data_as(ctypes.c_void_p)))
+    return anchors.tolist(), nearest.tolist()
 
 
 @dataclass
@@ -235,18 +237,21 @@ class AnchorPlan:
 
 
 def anchor_plan(frames, rows, cols, k_anchor, Np, device):
-    """Plan of :func:`anchor_attention` for a frames x rows x cols video padded to Np tokens."""
-    N = frames * rows * cols
-    anchors, nearest = anchor_rows(rows, k_anchor)
-    slot = {a: i for i, a in enumerate(anchors)}
-    fr = rows * cols
-    idx_q = [f * fr + a * cols + c for f in range(frames) for a in anchors for c in range(cols)]
-    nq = len(idx_q)
-    npq = (nq + 127) // 128 * 128
-    per_frame = len(anchors) * cols
-    idx_o = [f * per_frame + slot[nearest[r]] * cols + c for f in range(frames) for r in range(rows) for c in range(cols)]
-    as_dev = lambda x: torch.tensor(x, dtype=torch.int32, device=device)
-    return AnchorPlan(N, Np, nq, npq, as_dev(idx_q + [-1] * (npq - nq)), as_dev(idx_o + [-1] * (Np - N)))
+    """Plan of :func:`anchor_attention` for a frames x rows x cols video padded
+    to Np tokens: ``calibatt_anchor_plan`` on the device."""
+    lib = load()
+    nq, npq = ctypes.c_int(0), ctypes.c_int(0)
+    check(lib.calibatt_anchor_plan_size(int(frames), int(rows), int(cols), int(k_anchor), ctypes.byref(nq),
+                                        ctypes.byref(npq)))
+    device = torch.device(device)
+    if device.type != "cuda":
+        raise ValueError("the anchor plan is computed on a CUDA device")
+    idx_q = torch.empty(npq.value, dtype=torch.int32, device=device)
+    idx_o = torch.empty(int(Np), dtype=torch.int32, device=device)
+    with torch.cuda.device(device):
+        check(lib.calibatt_anchor_plan(int(frames), int(rows), int(cols), int(k_anchor), int(Np), _ptr(idx_q),
+                                       _ptr(idx_o), _stream(device)))
+    return AnchorPlan(int(frames) * int(rows) * int(cols), int(Np), nq.value, npq.value, idx_q, idx_o)
 
 
 def anchor_attention(q, k, v, plan: AnchorPlan, bl=None, scale=None):
@@ -447,39 +452,58 @@ def skiplist_report(masks, maps_per_layer, pcts=(100.0, 99.0, 95.0)):
     Per layer: full allocation (ceil(nkb / 2) intervals per row), trimmed to
     the widest row, and merged at each percentile in ``pcts`` (nearest rank of
     the layer's interval counts; outlier rows merged by
-    :func:`merge_intervals`, whose filled blocks lower the sparsity).  Host
-    arithmetic on the device's interval counts; synchronizes.
+    :func:`merge_intervals`, whose filled blocks lower the sparsity).  Sizes
+    from ``calibatt_skiplist_sizes`` and ``calibatt_blocklist_bytes``;
+    synchronizes.
     """
+    lib = load()
     n_maps, nqb, nkb = masks.shape
-    counts = interval_counts(masks).cpu()
     if n_maps % maps_per_layer:
         raise ValueError("n_maps must be a multiple of maps_per_layer")
+    dev = masks.device
+    counts = interval_counts(masks)
     layers = n_maps // maps_per_layer
-    rows_per_layer = maps_per_layer * nqb
-    per_layer = counts.view(layers, rows_per_layer).to(torch.int64)
-    full = layers * rows_per_layer * ((nkb + 1) // 2) * 8
-    trimmed = int(per_layer.max(dim=1).values.sum()) * rows_per_layer * 8
-    kept = int((masks != 0).sum())
-    out = {"rows": n_maps * nqb, "kept_blocks": kept, "density": kept / float(n_maps * nqb * nkb),
-           "intervals_max": int(counts.max()), "intervals_p95": _nearest_rank(counts, 95.0),
-           "skiplist_full_bytes": full, "skiplist_trimmed_bytes": trimmed, "merged": []}
-    for pct in pcts:
-        widths = [_nearest_rank(per_layer[l], pct) for l in range(layers)]
-        m = masks.clone()
-        filled = merge_intervals(m, [w for w in widths for _ in range(maps_per_layer)])
-        out["merged"].append({"pct": pct, "bytes": sum(widths) * rows_per_layer * 8, "filled_blocks": filled,
-                              "density": (kept + filled) / float(n_maps * nqb * nkb)})
-        del m
+
+    def sizes(mpl, pc):
+        nl = n_maps // mpl
+        n = ctypes.c_size_t(0)
+        check(lib.calibatt_skiplist_sizes_workspace_size(n_maps, mpl, len(pc), ctypes.byref(n)))
+        ws = torch.empty(n.value, dtype=torch.uint8, device=dev)
+        pc_h = np.asarray(pc, dtype=np.float64)
+        layer_max = np.zeros(nl, dtype=np.int32)
+        layer_width = np.zeros(max(1, len(pc) * nl), dtype=np.int32)
+        map_width = torch.empty(max(1, len(pc) * n_maps), dtype=torch.int32, device=dev)
+        nbytes = np.zeros(2 + len(pc), dtype=np.int64)
+        with torch.cuda.device(dev):
+            check(lib.calibatt_skiplist_sizes(_ptr(counts), n_maps, nqb, nkb, mpl,
+                                              pc_h.ctypes.data_as(ctypes.c_void_p), len(pc),
+                                              layer_max.ctypes.data_as(ctypes.c_void_p),
+                                              layer_width.ctypes.data_as(ctypes.c_void_p), _ptr(map_width),
+                                              nbytes.ctypes.data_as(ctypes.c_void_p), _ptr(ws), ws.numel(),
+                                              _stream(dev)))
+        return layer_max, layer_width, map_width, nbytes
+
+    layer_max, layer_width, map_width, nbytes = sizes(maps_per_layer, pcts)
+    g_max, g_p95, _, _ = sizes(n_maps, (95.0,))   # the whole dictionary as one group: max and p95
     nnz, n_pat, nnz_pat = compile_size(masks)
-    out["csr_bytes"] = (n_maps * nqb + 1) * 8 + nnz * 2
-    out["pattern_pool_bytes"] = n_maps * nqb * 8 + (n_pat + 1) * 4 + nnz_pat * 2
+    cells = float(n_maps * nqb * nkb)
+    out = {"rows": n_maps * nqb, "kept_blocks": nnz, "density": nnz / cells,
+           "intervals_max": int(g_max[0]), "intervals_p95": int(g_p95[0]),
+           "skiplist_full_bytes": int(nbytes[0]), "skiplist_trimmed_bytes": int(nbytes[1]),
+           "layer_max": layer_max.tolist(), "merged": []}
+    for p, pct in enumerate(pcts):
+        m = masks.clone()
+        filled = merge_intervals(m, map_width[p * n_maps:(p + 1) * n_maps])
+        out["merged"].append({"pct": pct, "bytes": int(nbytes[2 + p]), "filled_blocks": filled,
+                              "layer_width": layer_width[p * layers:(p + 1) * layers].tolist(),
+                              "density": (nnz + filled) / cells})
+        del m
+    csr, pool = ctypes.c_int64(0), ctypes.c_int64(0)
+    check(lib.calibatt_blocklist_bytes(n_maps, nqb, int(nnz), int(n_pat), int(nnz_pat), ctypes.byref(csr),
+                                       ctypes.byref(pool)))
+    out["csr_bytes"] = csr.value
+    out["pattern_pool_bytes"] = pool.value
     return out
-
-
-def _nearest_rank(values, pct):
-    v = torch.sort(values.reshape(-1).to(torch.int64)).values
-    k = max(1, math.ceil(pct / 100.0 * v.numel()))
-    return int(v[k - 1])
 
 
 def calibrate_schedule(inputs_per_step, N, param_of, select_mode=SELECT_ENERGY, rho=0.5, **kw):

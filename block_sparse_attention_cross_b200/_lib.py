@@ -70,6 +70,14 @@ EXPORTS = {
     "calibatt_compile": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_size_t,
                                  c_void_p]),
     "calibatt_selftest_wait_timeout": (c_int, [c_uint64, c_void_p, c_void_p]),
+    "calibatt_anchor_rows": (c_int, [c_int, c_int, c_void_p, c_void_p]),
+    "calibatt_anchor_plan_size": (c_int, [c_int, c_int, c_int, c_int, POINTER(c_int), POINTER(c_int)]),
+    "calibatt_anchor_plan": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "calibatt_skiplist_sizes_workspace_size": (c_int, [c_int, c_int, c_int, POINTER(c_size_t)]),
+    "calibatt_skiplist_sizes": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "calibatt_blocklist_bytes": (c_int, [c_int, c_int, c_int64, c_int32, c_int32, POINTER(c_int64),
+                                         POINTER(c_int64)]),
 }
 
 

@@ -206,6 +206,45 @@ int calibatt_gather_rows(const void* src, void* dst, const int32_t* idx, int n_p
                          int row_bytes, calibatt_stream_t stream);
 
 /*
+ * calibatt_anchor_rows -- the anchor rows of the spatial-repetition path
+ * (paper page, Figure 5(b) bottom: attention is computed for k anchor query
+ * rows per frame and broadcast to the neighbouring rows; Table S4: k of the
+ * 30 spatial rows at 480p).  Host arithmetic only (no device work).
+ *  anchors  host int32 [k] (written): anchor i = floor((i + 1/2) rows / k),
+ *           evenly spaced and centred, ascending;
+ *  nearest  host int32 [rows] (written): the anchor row every spatial row takes
+ *           its output from (the nearest anchor, the lower one on a tie).
+ * Errors: CALIBATT_E_INVALID unless 1 <= k <= rows and both pointers are set.
+ */
+int calibatt_anchor_rows(int rows, int k, int32_t* anchors, int32_t* nearest);
+
+/*
+ * calibatt_anchor_plan_size -- the gathered query count of the
+ * spatial-repetition path for a frames x rows x cols video: nq = frames k cols
+ * anchor tokens, padded to npq (a multiple of 128).  Host arithmetic only.
+ * Errors: CALIBATT_E_INVALID for a bad geometry or k outside [1, rows].
+ */
+int calibatt_anchor_plan_size(int frames, int rows, int cols, int k, int* nq, int* npq);
+
+/*
+ * calibatt_anchor_plan -- the two index lists of the spatial-repetition path
+ * (paper page, Figure 4 and Figure 5(b) bottom), computed on the device:
+ *  idx_q  device int32 [npq] (written): idx_q[i] = token of gathered query i
+ *         (anchor tokens ordered by frame, anchor, column); -1 for i >= nq;
+ *  idx_o  device int32 [Np] (written): idx_o[t] = gathered row whose output
+ *         video token t takes (same frame and column, nearest anchor row);
+ *         -1 for t >= frames rows cols.
+ * Use: q_anchor = gather(q, idx_q); O_anchor = forward(q_anchor, k, v) with
+ * calibatt_sparse_attn_fwd_qk; O = gather(O_anchor, idx_o)
+ * (calibatt_gather_rows).  Asynchronous on `stream`.
+ * Errors: as calibatt_anchor_plan_size; CALIBATT_E_INVALID if an index list
+ * is NULL or Np is below the video token count.
+ */
+int calibatt_anchor_plan(int frames, int rows, int cols, int k, int Np, int32_t* idx_q, int32_t* idx_o,
+                         calibatt_stream_t stream);
+
+
+/*
  * calibatt_block_energy -- block energies of one calibration input.
  *
  * Paper page, Figure 2 (block-level post-softmax attention maps) and
@@ -383,6 +422,49 @@ int calibatt_interval_counts(const uint8_t* masks, int n_maps, int nqb, int nkb,
  */
 int calibatt_merge_intervals(uint8_t* masks, int n_maps, int nqb, int nkb, const int32_t* width,
                              unsigned long long* filled, calibatt_stream_t stream);
+
+/*
+ * calibatt_skiplist_sizes -- sizes of the paper page's padded per-layer
+ * interval skip lists (Figure S10, Table S3) from the interval counts of a
+ * mask dictionary (calibatt_interval_counts).  A layer is maps_per_layer
+ * consecutive maps (all of its timesteps and heads); its array has one row per
+ * (map, query block) and one slot per interval (an int32 pair, 8 bytes):
+ *  full     ceil(nkb / 2) slots per row (the most a row can need);
+ *  trimmed  the layer's largest count (layer_max);
+ *  merged   for each percentile pcts[p] in (0, 100], the nearest-rank
+ *           percentile of the layer's counts: the smallest count c such that
+ *           at least ceil(pcts[p] / 100 * rows) counts are <= c
+ *           (layer_width); rows above it are merged to it with
+ *           calibatt_merge_intervals, which fills their smallest gaps.
+ *  counts       device int32 [n_maps * nqb];
+ *  layer_max    host int32 [n_layers] (written), n_layers = n_maps / maps_per_layer;
+ *  layer_width  host int32 [n_pcts * n_layers] (written), percentile-major;
+ *  map_width    device int32 [n_pcts * n_maps] (written) or NULL: each map's
+ *               layer width per percentile, the width argument of
+ *               calibatt_merge_intervals (map_width + p * n_maps);
+ *  bytes        host int64 [2 + n_pcts] (written): full, trimmed, then merged
+ *               for each percentile;
+ *  workspace    device, >= calibatt_skiplist_sizes_workspace_size bytes.
+ * Synchronizes `stream`.  nkb <= 16384, n_pcts <= 64.
+ * Errors: CALIBATT_E_INVALID for bad sizes or percentiles, CALIBATT_E_WORKSPACE
+ * for a short workspace, CALIBATT_E_CUDA if a copy fails.
+ */
+int calibatt_skiplist_sizes_workspace_size(int n_maps, int maps_per_layer, int n_pcts, size_t* bytes);
+int calibatt_skiplist_sizes(const int32_t* counts, int n_maps, int nqb, int nkb, int maps_per_layer,
+                            const double* pcts, int n_pcts, int32_t* layer_max, int32_t* layer_width,
+                            int32_t* map_width, int64_t* bytes, void* workspace, size_t workspace_bytes,
+                            calibatt_stream_t stream);
+
+/*
+ * calibatt_blocklist_bytes -- bytes of this library's compiled forms of a
+ * mask dictionary, for comparison with the skip lists: the plain CSR (int64
+ * row pointers, int16 columns) and the pattern pool (int32 base and pattern
+ * id per row, int32 pattern pointers, int16 offsets); sizes from
+ * calibatt_compile_size.  Host arithmetic only.
+ */
+int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, int32_t nnz_pat, int64_t* csr_bytes,
+                             int64_t* pool_bytes);
+
 
 /*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the

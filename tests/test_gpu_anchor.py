@@ -30,6 +30,32 @@ def test_gather_rows_exact():
     assert torch.equal(got, want)
 
 
+@pytest.mark.parametrize("frames,rows,cols,k", [(3, 7, 5, 3), (21, 30, 52, 5), (21, 30, 52, 30), (21, 45, 80, 4),
+                                                 (2, 6, 5, 1)])
+def test_anchor_plan_matches_the_oracle_mapping(frames, rows, cols, k):
+    # calibatt_anchor_plan on the device, bit for bit: gathered query i is the
+    # token of its frame's anchor row, every token's output comes from the
+    # gathered row of the token on its nearest anchor row, padding is -1.
+    N = frames * rows * cols
+    Np = (N + 127) // 128 * 128
+    plan = cba.anchor_plan(frames, rows, cols, k, Np, "cuda")
+    anchors, nearest = oracle.anchor_rows(rows, k)
+    per_frame = k * cols
+    want_q = np.full(plan.npq, -1, np.int64)
+    want_o = np.full(Np, -1, np.int64)
+    for f in range(frames):
+        for a, ar in enumerate(anchors):
+            for c in range(cols):
+                want_q[f * per_frame + a * cols + c] = (f * rows + ar) * cols + c
+        for r in range(rows):
+            slot = anchors.index(nearest[r])
+            for c in range(cols):
+                want_o[(f * rows + r) * cols + c] = f * per_frame + slot * cols + c
+    assert plan.nq == frames * k * cols and plan.npq % 128 == 0 and plan.npq - plan.nq < 128
+    assert np.array_equal(plan.idx_q.cpu().numpy(), want_q)
+    assert np.array_equal(plan.idx_o.cpu().numpy(), want_o)
+
+
 @pytest.mark.parametrize("k_anchor", [10, 4, 1])
 def test_anchor_attention_small_video(k_anchor):
     frames, rows, cols, H, d = 3, 10, 20, 2, 128

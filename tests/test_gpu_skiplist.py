@@ -34,6 +34,35 @@ def test_counts_and_merge_match_oracle():
     assert (oracle.interval_counts(want) <= np.maximum(width, 1)[:, None]).all()
 
 
+@pytest.mark.parametrize("maps_per_layer,pcts", [(3, (100.0, 99.0, 95.0, 50.0)), (12, (95.0, 12.5)), (1, (100.0,))])
+def test_skiplist_sizes_match_the_oracle(maps_per_layer, pcts):
+    # calibatt_skiplist_sizes: per-layer maximum and nearest-rank percentile
+    # widths of the interval counts and the byte totals, bit for bit against
+    # the oracle; the per-map widths drive the merge to the oracle's masks.
+    rng = np.random.default_rng(9)
+    n_maps, nqb, nkb = 12, 9, 75
+    dens = rng.choice([0.05, 0.2, 0.5, 0.9], size=(n_maps, nqb, 1))
+    masks = (rng.random((n_maps, nqb, nkb)) < dens).astype(np.uint8)
+    md = torch.from_numpy(masks).cuda()
+    rep = cba.skiplist_report(md, maps_per_layer, pcts)
+    counts = oracle.interval_counts(masks)
+    layers = n_maps // maps_per_layer
+    per_layer = counts.reshape(layers, -1)
+    assert rep["layer_max"] == per_layer.max(axis=1).tolist()
+    assert rep["intervals_max"] == int(counts.max()) and rep["intervals_p95"] == oracle.nearest_rank(counts, 95.0)
+    for m, pct in zip(rep["merged"], pcts):
+        want = oracle.skiplist_bytes(counts, maps_per_layer, nkb, pct=pct)
+        assert (rep["skiplist_full_bytes"], rep["skiplist_trimmed_bytes"], m["bytes"]) == \
+            (want["full"], want["trimmed"], want["merged"])
+        widths = [oracle.nearest_rank(per_layer[l], pct) for l in range(layers)]
+        assert m["layer_width"] == widths
+        merged = oracle.merge_masks(masks, np.repeat(widths, maps_per_layer))
+        assert m["filled_blocks"] == int(merged.sum()) - int(masks.sum())
+    bl = oracle.compile_blocklist(masks)
+    assert rep["csr_bytes"] == (n_maps * nqb + 1) * 8 + int(masks.sum()) * 2
+    assert rep["pattern_pool_bytes"] == n_maps * nqb * 8 + bl["pat_ptr"].size * 4 + bl["pat_off"].size * 2
+
+
 def _report(masks_np, maps_per_layer, name):
     md = torch.from_numpy(masks_np).cuda()
     assert np.array_equal(cba.interval_counts(md).cpu().numpy(), oracle.interval_counts(masks_np))

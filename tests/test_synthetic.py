@@ -79,23 +79,19 @@ def test_video_qkv_shapes_and_padding():
     assert c > 0.9
 
 
-def test_anchor_plan_indices_match_the_oracle_mapping():
-    # The host-side index lists of the spatial-repetition path: gathered query
-    # i is the token of anchor row a(i) of its frame, and every token's output
-    # comes from the gathered row of the token on its nearest anchor row.
+def test_anchor_rows_through_the_c_abi_match_the_oracle():
+    # calibatt_anchor_rows is host arithmetic in the library (no device work):
+    # anchors and nearest-anchor mapping equal the oracle's for every k of the
+    # pages' 30-row frames and for odd small frames; sizes of the gathered
+    # query tensor follow the geometry.
+    import ctypes
     import oracle
     import block_sparse_attention_cross_b200 as cba
-    frames, rows, cols, k = 3, 7, 5, 3
-    N = frames * rows * cols
-    Np = (N + 127) // 128 * 128
-    plan = cba.anchor_plan(frames, rows, cols, k, Np, "cpu")
-    anchors, nearest = oracle.anchor_rows(rows, k)
-    assert (anchors, nearest) == cba.anchor_rows(rows, k)
-    iq = plan.idx_q.tolist()
-    io = plan.idx_o.tolist()
-    assert plan.nq == frames * k * cols and plan.npq % 128 == 0 and len(iq) == plan.npq
-    assert all(x == -1 for x in iq[plan.nq:]) and all(x == -1 for x in io[N:])
-    for t in range(N):
-        f, rem = divmod(t, rows * cols)
-        r, c = divmod(rem, cols)
-        assert iq[io[t]] == f * rows * cols + nearest[r] * cols + c
+    for rows in (30, 45, 7, 1):
+        for k in range(1, rows + 1):
+            assert cba.anchor_rows(rows, k) == oracle.anchor_rows(rows, k)
+    lib = cba.load()
+    nq, npq = ctypes.c_int(0), ctypes.c_int(0)
+    assert lib.calibatt_anchor_plan_size(21, 30, 52, 5, ctypes.byref(nq), ctypes.byref(npq)) == 0
+    assert (nq.value, npq.value) == (21 * 5 * 52, 5504)
+    assert lib.calibatt_anchor_plan_size(2, 30, 52, 31, ctypes.byref(nq), ctypes.byref(npq)) == cba._lib.E_INVALID
