@@ -30,7 +30,8 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
 __all__ = [
     "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
     "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "gather_rows",
-    "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "calibrate_schedule", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
+    "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "spatial_similarity", "repetition_flags",
+    "calibrate_schedule", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
@@ -278,6 +279,43 @@ def anchor_attention(q, k, v, plan: AnchorPlan, bl=None, scale=None):
                                                  int(plan.N), Np, d, _dtype_code(q), scale, ctypes.byref(s), 0, None,
                                                  _stream(q.device)))
     return gather_rows(og, plan.idx_o)
+
+
+def spatial_similarity(q, k, N, frames, rows, cols, scale=None, status=None):
+    """Spatial-similarity score [H] float32 of one input (``calibatt_spatial_similarity``).
+
+    q, k: [H, Np, d] bf16 CUDA tensors; the first frames x rows x cols tokens
+    are the video.  The score of a head is the mean cosine similarity of the
+    dense attention rows of vertically adjacent query tokens (same frame and
+    column): near 1 for maps that repeat across spatial rows (paper page,
+    Figure 4, Figure 6(a), Figure S13).
+    """
+    _need_cuda(q, k)
+    H, Np, d = q.shape
+    scale = default_scale(d) if scale is None else float(scale)
+    n = ctypes.c_size_t(0)
+    check(load().calibatt_spatial_similarity_workspace_size(H, Np, ctypes.byref(n)))
+    ws = torch.empty(n.value, dtype=torch.uint8, device=q.device)
+    out = torch.empty(H, dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        check(load().calibatt_spatial_similarity(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), int(frames),
+                                                 int(rows), int(cols), scale, _ptr(out), _ptr(ws), ws.numel(),
+                                                 _ptr(status), _stream(q.device)))
+    return out
+
+
+def repetition_flags(scores, tau=0.87):
+    """Repetition dictionary (``calibatt_repetition_flags``): from per-input
+    scores [n_inputs, n_maps] float32 (CUDA), the mean score per map and the
+    flags mean >= tau (paper page, Figure 5(a), Figure S13: tau = 0.87)."""
+    _need_cuda(scores)
+    n_inputs, n_maps = scores.shape
+    mean = torch.empty(n_maps, dtype=torch.float32, device=scores.device)
+    flags = torch.empty(n_maps, dtype=torch.uint8, device=scores.device)
+    with torch.cuda.device(scores.device):
+        check(load().calibatt_repetition_flags(_ptr(scores), n_inputs, n_maps, float(tau), _ptr(mean), _ptr(flags),
+                                               _stream(scores.device)))
+    return mean, flags
 
 
 def _calib_workspace(H, N, Np, d, bq, bk, device):

@@ -78,6 +78,10 @@ EXPORTS = {
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "calibatt_blocklist_bytes": (c_int, [c_int, c_int, c_int64, c_int32, c_int32, POINTER(c_int64),
                                          POINTER(c_int64)]),
+    "calibatt_spatial_similarity_workspace_size": (c_int, [c_int, c_int, POINTER(c_size_t)]),
+    "calibatt_spatial_similarity": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                            c_int, c_float, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "calibatt_repetition_flags": (c_int, [c_void_p, c_int, c_int, c_float, c_void_p, c_void_p, c_void_p]),
 }
 
 

@@ -20,7 +20,7 @@ INCLUDE = PKG.parent / "include"
 BUILD = PKG / "_build"
 LIB = PKG / "libcalibatt.so"
 
-SOURCES = ["api.cu", "attn_tc.cu", "attn_fwd.cu", "attn_simt.cu", "select_vote.cu", "compile.cu", "noalloc.cu", "sharing.cu", "skiplist.cu", "gather.cu", "plan.cu"]
+SOURCES = ["api.cu", "attn_tc.cu", "attn_fwd.cu", "attn_simt.cu", "select_vote.cu", "compile.cu", "noalloc.cu", "sharing.cu", "skiplist.cu", "gather.cu", "plan.cu", "similarity.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 NVCC_FLAGS = [

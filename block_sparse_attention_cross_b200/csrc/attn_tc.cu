@@ -267,6 +267,16 @@ int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const TcArgs& a, di
 
 }  // namespace
 
+int launch_tc_stats(const void* q, const void* k, int d, const TcArgs& a, cudaStream_t s) {
+  CUtensorMap tq, tk;
+  const uint64_t rows = static_cast<uint64_t>(a.H) * a.Np;
+  int rc;
+  if ((rc = make_tmap_bf16(&tq, q, rows, d)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tk, k, rows, d)) != CALIBATT_OK) return rc;
+  dim3 grid(a.nqb, a.H, 1);
+  return d == 128 ? launch_one<128, MODE_STATS>(tq, tk, a, grid, s) : launch_one<64, MODE_STATS>(tq, tk, a, grid, s);
+}
+
 int launch_tc_energy(const void* q, const void* k, int d, const TcArgs& a, cudaStream_t s) {
   CUtensorMap tq, tk;
   const uint64_t rows = static_cast<uint64_t>(a.H) * a.Np;

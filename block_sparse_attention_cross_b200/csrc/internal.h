@@ -65,6 +65,8 @@ int energy_impl(const void* q, const void* k, int H, int N, int Np, int d, int d
 // attn_tc.cu (bf16, tcgen05)
 int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcArgs& a, cudaStream_t s);
 int launch_tc_energy(const void* q, const void* k, int d, const TcArgs& a, cudaStream_t s);
+// The STATS pass alone: a.lse2[h * Np + row] = log2-domain LSE of every row over the real keys.
+int launch_tc_stats(const void* q, const void* k, int d, const TcArgs& a, cudaStream_t s);
 
 // attn_simt.cu (fp32, FFMA)
 int launch_simt_fwd(const void* q, const void* k, const void* v, void* o, int d, const SimtArgs& a,

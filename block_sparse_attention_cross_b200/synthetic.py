@@ -163,11 +163,13 @@ def _token_coords(grid: VideoGrid):
     return f, y, x
 
 
-def video_qk_base(grid: VideoGrid, H, d, seed, rank=16, alpha=1.0, jitter=0.0, jitter_seed=None):
+def video_qk_base(grid: VideoGrid, H, d, seed, rank=16, alpha=1.0, jitter=0.0, jitter_seed=None, row_scale=None):
     """Shared low-rank frame/row/column structure: [H, video_tokens, d] float32.
 
-    base[h, t] = alpha * (F[h, f(t)] + Y[h, y(t)] + X[h, x(t)]) @ W[h], with
-    F, Y, X ~ N(0, 1) of width ``rank`` and W ~ N(0, 1/rank).  ``jitter`` adds
+    base[h, t] = alpha * (F[h, f(t)] + s_h Y[h, y(t)] + X[h, x(t)]) @ W[h], with
+    F, Y, X ~ N(0, 1) of width ``rank`` and W ~ N(0, 1/rank); s_h =
+    ``row_scale[h]`` (1 when not given: heads whose s_h is small see nearly the
+    same tokens on every spatial row of a frame).  ``jitter`` adds
     N(0, jitter^2) to F, Y and X from ``jitter_seed`` (per calibration input).
     """
     rng = np.random.default_rng(seed)
@@ -183,8 +185,10 @@ def video_qk_base(grid: VideoGrid, H, d, seed, rank=16, alpha=1.0, jitter=0.0, j
     f, y, x = _token_coords(grid)
     base = np.empty((H, grid.video_tokens, d), dtype=np.float32)
 
+    rs = np.ones(H) if row_scale is None else np.asarray(row_scale, np.float64)
+
     def head(h):
-        lat = F[h][f] + Y[h][y] + X[h][x]
+        lat = F[h][f] + rs[h] * Y[h][y] + X[h][x]
         base[h] = (alpha * (lat @ W[h])).astype(np.float32)
 
     with ThreadPoolExecutor(_threads()) as ex:
@@ -192,7 +196,7 @@ def video_qk_base(grid: VideoGrid, H, d, seed, rank=16, alpha=1.0, jitter=0.0, j
     return base
 
 
-def video_qkv(w: Workload, noise=0.1, with_v=True, input_index=None, jitter=0.05):
+def video_qkv(w: Workload, noise=0.1, with_v=True, input_index=None, jitter=0.05, row_scale=None):
     """Q, K (and V) float32 [B, H, Np, d] for a video-shaped workload.
 
     Q and K share the low-rank base and get independent N(0, noise^2) noise;
@@ -201,15 +205,17 @@ def video_qkv(w: Workload, noise=0.1, with_v=True, input_index=None, jitter=0.05
     from seeds derived from 100 + n (calibration inputs).  Every (tensor,
     batch, head) slice draws from its own stream, seeded by (seed, b, h), so
     the slices are filled in parallel and the values do not depend on the
-    thread count.
+    thread count.  ``row_scale``: per-head weight of the spatial-row term of
+    the base (see :func:`video_qk_base`).
     """
     g = w.grid
     s = w.seeds
     if input_index is None:
-        base = video_qk_base(g, w.H, w.d, s["base"])
+        base = video_qk_base(g, w.H, w.d, s["base"], row_scale=row_scale)
         sq, sk = [s["noise_q"]], [s["noise_k"]]
     else:
-        base = video_qk_base(g, w.H, w.d, s["base"], jitter=jitter, jitter_seed=100 + input_index)
+        base = video_qk_base(g, w.H, w.d, s["base"], jitter=jitter, jitter_seed=100 + input_index,
+                             row_scale=row_scale)
         sq, sk = [100 + input_index, 1], [100 + input_index, 2]
     sv = [s.get("v", 0)]
     Nv, N, Np = g.video_tokens, w.N, w.Np

@@ -243,6 +243,50 @@ int calibatt_anchor_plan_size(int frames, int rows, int cols, int k, int* nq, in
 int calibatt_anchor_plan(int frames, int rows, int cols, int k, int Np, int32_t* idx_q, int32_t* idx_o,
                          calibatt_stream_t stream);
 
+/*
+ * calibatt_spatial_similarity -- the spatial-similarity score of every head's
+ * attention map for one input (paper page, Figure 4: the attention pattern
+ * repeats across the spatial rows of a frame; Figure 6(a) plots a map's
+ * "spatial similarity"; Figure S13 flags heads whose score exceeds
+ * tau = 0.87).  The pages do not define the score; this library reads it as
+ * the mean, over the video query tokens (f, r, c) with r < rows - 1, of the
+ * cosine similarity between the dense attention rows (softmax over all N real
+ * keys) of tokens (f, r, c) and (f, r + 1, c), the two rows the anchor
+ * broadcast (Figure 5(b) bottom) would give the same output.  Rows of P are
+ * non-negative, so scores lie in [0, 1].
+ *  q, k       [H, Np, d] bf16 device; tokens t < frames rows cols are the video
+ *             (t = (f rows + r) cols + c), any further real tokens (< N, e.g.
+ *             text) are keys only;
+ *  score_out  [H] float32 device (written);
+ *  workspace  device, >= calibatt_spatial_similarity_workspace_size bytes.
+ * bf16, d in {64, 128}; N, Np as calibatt_block_energy; rows >= 2.
+ * Deterministic (fixed-order reductions); asynchronous on `stream`.
+ * Errors: CALIBATT_E_INVALID / E_UNSUPPORTED / E_WORKSPACE as the other calls
+ * (nothing launched); device timeouts go to dev_status.
+ */
+int calibatt_spatial_similarity_workspace_size(int H, int Np, size_t* bytes);
+int calibatt_spatial_similarity(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int frames,
+                                int rows, int cols, float scale, float* score_out, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, calibatt_stream_t stream);
+
+/*
+ * calibatt_repetition_flags -- the repetition dictionary (paper page, Figure
+ * 5(a): heads that show spatial row repetition are stored in a dictionary;
+ * Figure 6(b): the score varies little across calibration prompts; Figure
+ * S13: tau = 0.87): per map, the mean score over the calibration inputs and
+ * the flag mean >= tau.
+ *  scores     [n_inputs, n_maps] float32 device (one calibatt_spatial_similarity
+ *             per input, map id = (l T + t) H + h);
+ *  mean_out   [n_maps] float32 device (written; may be NULL): the float32 sum
+ *             in input order divided by n_inputs;
+ *  flags_out  [n_maps] uint8 device (written): 1 where mean >= tau.
+ * Asynchronous.  Errors: CALIBATT_E_INVALID for NULL pointers, bad sizes or a
+ * non-finite tau.
+ */
+int calibatt_repetition_flags(const float* scores, int n_inputs, int n_maps, float tau, float* mean_out,
+                              uint8_t* flags_out, calibatt_stream_t stream);
+
+
 
 /*
  * calibatt_block_energy -- block energies of one calibration input.

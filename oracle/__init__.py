@@ -30,6 +30,9 @@ blocking, fusion or reordering beyond what the definition states):
 * ``anchor_rows`` / ``anchor_attention`` -- spatial repetition: attention of
   k anchor rows per frame broadcast to the other rows (Figure 4, Figure 5(b)
   bottom, Table S4).
+* ``spatial_similarity`` / ``repetition_flags`` -- the per-head spatial
+  similarity score and the repetition dictionary (Figure 5(a), Figure 6,
+  Figure S13; the score's definition is this build's reading).
 * ``compile_blocklist`` / ``expand_blocklist`` -- compile masks into per-row
   kept-block lists with translation-relative row-pattern dedup (Abstract:
   "compiles these patterns into optimized attention operations for each
@@ -48,7 +51,7 @@ from .calibration import block_energy, block_energy_row, select_topk, select_ene
 from .compile import compile_blocklist, expand_blocklist
 from .sharing import skipped_iou, timestep_similarity, timestep_clusters, share_masks
 from .skiplist import interval_counts, merge_row, merge_masks, nearest_rank, skiplist_bytes
-from .anchor import anchor_rows, anchor_attention, anchor_attention_tokens
+from .anchor import anchor_rows, anchor_attention, anchor_attention_tokens, spatial_similarity, repetition_flags
 
 __all__ = [
     "masked_attention",

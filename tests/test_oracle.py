@@ -520,3 +520,56 @@ def test_block_energy_row_is_a_row_of_block_energy():
     E = oracle.block_energy(q, k, N, 128, 64, 0.25)
     for h, qb in ((0, 0), (1, 2), (1, 1)):
         assert np.array_equal(oracle.block_energy_row(q, k, N, 128, 64, 0.25, h, qb), E[h, qb])
+
+
+def _sim_video(frames, rows, cols, text, d, rng, same_rows=False):
+    N = frames * rows * cols + text
+    q = rng.standard_normal((2, N + 3, d))
+    if same_rows:   # every spatial row of a frame repeats the first one (per frame and column)
+        for f in range(frames):
+            for r in range(1, rows):
+                q[:, (f * rows + r) * cols:(f * rows + r + 1) * cols] = q[:, f * rows * cols:(f * rows + 1) * cols]
+    k = rng.standard_normal((2, N + 3, d))
+    return q, k, N
+
+
+def test_spatial_similarity_closed_forms():
+    rng = np.random.default_rng(31)
+    # rows that repeat within each frame (and differ across frames and columns): score 1
+    q, k, N = _sim_video(3, 4, 5, 7, 6, rng, same_rows=True)
+    assert np.allclose(oracle.spatial_similarity(q, k, N, 3, 4, 5, 0.7), 1.0, atol=1e-12)
+    # one-hot attention on distinct keys: neighbouring rows share nothing, score 0
+    frames, rows, cols = 2, 3, 4
+    n = frames * rows * cols
+    e = np.eye(n)[None].repeat(2, axis=0) * 40.0
+    assert np.allclose(oracle.spatial_similarity(e, e, n, frames, rows, cols, 1.0), 0.0, atol=1e-12)
+
+
+def test_spatial_similarity_brute_force():
+    rng = np.random.default_rng(32)
+    frames, rows, cols, text, d, scale = 2, 3, 2, 2, 4, 0.6
+    q, k, N = _sim_video(frames, rows, cols, text, d, rng)
+    got = oracle.spatial_similarity(q, k, N, frames, rows, cols, scale)
+    for h in range(2):
+        def prow(t):
+            s = [scale * sum(q[h, t, x] * k[h, j, x] for x in range(d)) for j in range(N)]
+            m = max(s)
+            e = [math.exp(v - m) for v in s]
+            z = math.fsum(e)
+            return [v / z for v in e]
+        cos = []
+        for f in range(frames):
+            for r in range(rows - 1):
+                for c in range(cols):
+                    a = prow((f * rows + r) * cols + c)
+                    b = prow((f * rows + r + 1) * cols + c)
+                    num = math.fsum(x * y for x, y in zip(a, b))
+                    den = math.sqrt(math.fsum(x * x for x in a) * math.fsum(y * y for y in b))
+                    cos.append(num / den)
+        assert abs(got[h] - math.fsum(cos) / len(cos)) < 1e-12
+
+
+def test_repetition_flags_hand_case():
+    scores = np.array([[1.0, 0.5, 0.75], [0.5, 0.5, 1.0]], np.float32)
+    mean, flags = oracle.repetition_flags(scores, 0.75)
+    assert mean.tolist() == [0.75, 0.5, 0.875] and flags.tolist() == [1, 0, 1]
