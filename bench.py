@@ -24,7 +24,9 @@ At N = 1 the line also carries a ``workloads`` record with the other
 configurations, each timed on the device and checked against the float64
 oracle on a sample: the Wan 720p and Mochi calls (20% kept), the sweep of
 120 calls (40 layers x 3 timesteps x 40 heads), one calibration pass of 8
-Wan 480p inputs, and the tiny fp32 case.
+Wan 480p inputs, the Wan 480p call with each key-block size of the paper
+page's Table S6 (64 ... 144 keys) at its reported sparsity, and the tiny
+fp32 case.
 
 ``--gpus N`` without a launcher starts N replica processes itself (one per
 GPU, the torchrun environment set for each); under torchrun the world size
@@ -548,6 +550,52 @@ def _tiny_fp32_workload(device):
                                     "within_bound": bool(err.max() <= 1e-5)}}
 
 
+TABLE_S6_DENSITY = {64: 0.351, 80: 0.354, 96: 0.359, 128: 0.366, 144: 0.369}   # 1 - sparsity, paper page Table S6
+
+
+def _key_block_workload(device, pk):
+    """The Wan 480p call with each key-block size of the paper page's Table S6
+    (B_q = 128, B_kv = 64 ... 144) at the sparsity the table reports: the
+    128 x 128 structured mask regridded to the key block, keys padded to a
+    multiple of the key block (calibatt_sparse_attn_fwd_qk)."""
+    import torch
+    import block_sparse_attention_cross_b200 as cba
+    from block_sparse_attention_cross_b200 import synthetic as syn
+    import oracle
+    w = workload(None, "wan480_25")
+    (q, k, v), host = _qkv_device(w, device)
+    scale = cba.default_scale(w.d)
+    out = torch.empty_like(q)
+    rec = {}
+    for bk, dens in TABLE_S6_DENSITY.items():
+        mask = syn.regrid_key_blocks(syn.workload_mask(w, density=dens), w.N, bk, dens, 17)
+        npk = mask.shape[2] * bk
+        kp = torch.zeros((1, w.H, npk, w.d), dtype=q.dtype, device=device)
+        vp = torch.zeros_like(kp)
+        kp[:, :, :w.N] = k[:, :, :w.N]
+        vp[:, :, :w.N] = v[:, :, :w.N]
+        bl = cba.compile(torch.from_numpy(mask).to(device), block_q=128, block_k=bk)
+        tot, _ = time_calls(lambda: cba.sparse_attn_fwd_qk(q, kp, vp, bl, w.N, w.N, out=out), 10, 3, torch)
+        ms = tot / 10
+        cba.sparse_attn_fwd_qk(q, kp, vp, bl, w.N, w.N, out=out)
+        torch.cuda.synchronize()
+        kh = np.zeros((1, w.H, npk, w.d), np.float32)
+        vh = np.zeros_like(kh)
+        kh[:, :, :w.N] = host[1][:, :, :w.N]
+        vh[:, :, :w.N] = host[2][:, :, :w.N]
+        errs = []
+        for h, qb in ((0, 0), (w.H - 1, w.nqb - 1), (17, 101)):
+            o, _ = oracle.masked_attention_rows(host[0][:, h:h + 1].astype(np.float64), kh[:, h:h + 1], vh[:, h:h + 1],
+                                                mask[h:h + 1], w.N, 128, bk, scale, 0, 0, qb)
+            errs.append(np.abs(out[0, h, qb * 128:(qb + 1) * 128].float().cpu().numpy().astype(np.float64) - o))
+        kept = kept_flops(bl.nnz, w.d, w.B, block_k=bk) / (ms / 1e3) / 1e12
+        rec[f"128x{bk}"] = {"density": round(bl.density, 4), "ms_per_call": round(ms, 4), "kept_tflops": round(kept, 2),
+                            "frac_of_bf16_burst": round(kept / pk["bf16_burst"], 4),
+                            "parity_sampled": dict(_parity(errs), blocks=3)}
+        del kp, vp, bl
+    return rec
+
+
 def other_workloads(device, pk):
     """The configurations besides the headline call, each timed and sampled against the oracle (N = 1)."""
     import torch
@@ -556,6 +604,7 @@ def other_workloads(device, pk):
                      ("mochi_20", lambda: _fwd_workload("mochi_20", device, pk)),
                      ("sweep_4800_maps", lambda: _sweep_workload(device, pk)),
                      ("calibration_8_inputs", lambda: _calibration_workload(device)),
+                     ("key_blocks_table_s6", lambda: _key_block_workload(device, pk)),
                      ("tiny_fp32", lambda: _tiny_fp32_workload(device))):
         t0 = time.perf_counter()
         rec[name] = fn()

@@ -28,7 +28,7 @@ from ._lib import (BF16, DEDUP_HASH, DEDUP_HASH_WEAK, DEDUP_NONE, FP32, SELECT_E
                    CalibattError, check, load)
 
 __all__ = [
-    "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
+    "BlockList", "sparse_attn_fwd", "sparse_attn_fwd_qk", "sparse_attn_fwd_streamed", "block_energy", "timestep_clusters",
     "share_masks", "share_timesteps", "interval_counts", "merge_intervals", "skiplist_report", "gather_rows",
     "anchor_rows", "anchor_plan", "AnchorPlan", "anchor_attention", "spatial_similarity", "repetition_flags",
     "calibrate_schedule", "block_energy_noalloc", "select_vote", "finalize_mask", "calibrate",
@@ -154,6 +154,34 @@ def sparse_attn_fwd(q, k, v, bl: BlockList, N, scale=None, map_offset=0, return_
         check(load().calibatt_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, int(N), Np, d,
                                               _dtype_code(q), scale, ctypes.byref(s), int(map_offset),
                                               _ptr(status), _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def sparse_attn_fwd_qk(q, k, v, bl: BlockList, Nq, Nk, scale=None, map_offset=0, return_lse=False, out=None,
+                       lse=None, status=None):
+    """Block-sparse attention forward with separate query and key lengths (bf16).
+
+    q: [B, H, Npq, d] (Nq real rows); k, v: [B, H, Npk, d] (Nk real keys).
+    ``bl`` has n_q_blocks = Npq / 128 and n_k_blocks = Npk / block_k, so the
+    key padding follows the key-block size (any of 64, 80, 96, 128, 144)
+    independently of the query blocks.  Returns O [B, H, Npq, d] (and LSE).
+    """
+    _need_cuda(q, k, v)
+    B, H, Npq, d = q.shape
+    Npk = k.shape[2]
+    if k.shape != (B, H, Npk, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k, v must be [B, H, Npk, d] of q's dtype")
+    scale = default_scale(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, Npq), device=q.device, dtype=torch.float32)
+    _need_cuda(out, lse, status)
+    s = bl.as_struct()
+    with torch.cuda.device(q.device):
+        check(load().calibatt_sparse_attn_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, int(Nq), Npq,
+                                                 int(Nk), Npk, d, _dtype_code(q), scale, ctypes.byref(s),
+                                                 int(map_offset), _ptr(status), _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

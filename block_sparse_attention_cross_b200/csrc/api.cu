@@ -172,8 +172,11 @@ int check_fwd(const void* q, const void* k, const void* v, const void* o, int B,
   if (static_cast<long long>(B) * H * (Npq > Npk ? Npq : Npk) >= (1ll << 31))
     return set_error(CALIBATT_E_UNSUPPORTED, "B*H*Np must be below 2^31 rows");
   if (dtype == CALIBATT_BF16) {
-    if (!(d == 64 || d == 128) || bl->block_q != 128 || !(bl->block_k == 128 || bl->block_k == 64))
-      return set_error(CALIBATT_E_UNSUPPORTED, "bf16 path supports d in {64,128} with 128x128 or 128x64 blocks");
+    const int bk = bl->block_k;
+    if (!(d == 64 || d == 128) || bl->block_q != 128 || !(bk == 64 || bk == 80 || bk == 96 || bk == 128 || bk == 144))
+      return set_error(CALIBATT_E_UNSUPPORTED,
+                       "bf16 path supports d in {64,128}, 128-row query blocks and key blocks of 64, 80, 96, 128 "
+                       "or 144");
     if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
     return CALIBATT_OK;
   }
@@ -201,7 +204,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     a.scale_log2 = scale * 1.4426950408889634f;
     a.row_base = bl->row_base; a.row_pat = bl->row_pat; a.pat_ptr = bl->pat_ptr; a.pat_off = bl->pat_off;
     a.n_pat = bl->n_pat; a.nnz_pat = bl->nnz_pat; a.map_offset = map_offset;
-    a.kscale = 128 / bl->block_k;
+    a.block_k = bl->block_k;
     a.o = o; a.lse = lse; a.status = dev_status; a.spin_ns = spin_limit_ns();
     return launch_tc_fwd(q, k, v, d, a, s);
   }

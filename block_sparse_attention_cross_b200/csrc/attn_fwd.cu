@@ -6,10 +6,13 @@
 // kept-block list; only the kept K/V tiles are loaded (TMA) and multiplied
 // (tcgen05), so a skipped block costs neither bytes nor FLOPs.
 //
-// Templated on the head dim D (128 or 64) and the key-block size BK (128 or
-// 64; query blocks are always 128 rows; the paper page's Table S6 compares
-// key-block sizes).  The text below describes BK = 128; with BK = 64 every
-// key-column count halves (64-row K/V tiles, 32 columns per softmax half).
+// Templated on the head dim D (128 or 64) and the key-block size BK (64, 80,
+// 96, 128 or 144; query blocks are always 128 rows; the paper page's Table S6
+// compares these key-block sizes).  The text below describes BK = 128.  In
+// general the two softmax halves take W0 = BK / 2 rounded up to a multiple of
+// 16 key columns and BK - W0 (80 = 48 + 32, 144 = 80 + 64), so that each
+// half's probabilities feed whole PV K steps of 16 keys; score buffers are 128
+// TMEM columns apart (160 for BK = 144) and O follows them.
 //
 // Persistent CTA (one per SM, one query tile at a time), 12 warps:
 //   warps 0-3   softmax, key columns 0-63 of each block (warp w: rows 32w..32w+31)
@@ -51,6 +54,7 @@
 // its own copies and MMAs, frees TMEM and exits.
 #include <atomic>
 #include <cmath>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -79,7 +83,14 @@ struct FwdLayout {
   static constexpr uint32_t KBOX_BYTES = BK * 64 * 2;    // BK rows x 64 bf16
   static constexpr uint32_t Q_BYTES = TILE * D * 2;
   static constexpr uint32_t KV_BYTES = BK * D * 2;
-  static constexpr int RING = ((D == 128) ? 5 : 10) * (TILE / BK);
+  static constexpr int RING = 163840 / KV_BYTES;               // 160 KB of K/V tiles
+  // Key columns of the two softmax halves: the first a multiple of 16 (one
+  // PV K step), the second the rest; and the TMEM stride of a score buffer.
+  static constexpr int W0 = (BK / 2 + 15) / 16 * 16;
+  static constexpr int W1 = BK - W0;
+  static constexpr uint32_t SB = BK <= 128 ? 128 : (BK + 31) / 32 * 32;
+  static_assert(W1 >= 32 && W1 % 16 == 0 && 2 * SB + 128 <= 512, "key-block size");
+  static_assert(KV_BYTES % 1024 == 0 && KBOX_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned tiles");
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_RING = Q_BYTES;
   static constexpr uint32_t OFF_XCHG = OFF_RING + RING * KV_BYTES;   // float2 [2 slots][2 halves][128 rows]
@@ -102,6 +113,9 @@ struct FwdCtrl {
   int abort;
 };
 
+template <int V>
+using IntC = std::integral_constant<int, V>;
+
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 
@@ -116,7 +130,7 @@ struct TileList {
 // Reads and checks the kept-block list of work tile t.  Warp-collective: every
 // lane returns the same result, and every role evaluates the same data, so
 // all roles agree on n.
-__device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool report, int kscale) {
+__device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool report) {
   TileList tl;
   tl.bh = t / a.nqb;
   tl.qb = t - tl.bh * a.nqb;
@@ -146,13 +160,15 @@ __device__ __forceinline__ TileList tile_list(const TcArgs& a, int t, bool repor
   if (bad && report && lane == 0) report_status(a.status, CALIBATT_E_CORRUPT);
   tl.n = bad ? 0 : n;
   tl.p0 = p0;
-  // Walk order: start at the query tile's own (diagonal) block, or the first
-  // kept block after it, and wrap around.  For video attention the query's
-  // own block usually holds the row maximum, so later blocks rarely raise it.
+  // Walk order: start at the query tile's own (diagonal) block -- the key
+  // block holding its first token -- or the first kept block after it, and
+  // wrap around.  For video attention the query's own block usually holds
+  // the row maximum, so later blocks rarely raise it.
+  const int kb_diag = tl.qb * TILE / a.block_k;
   int below = 0;
   for (int i0 = 0; i0 < tl.n; i0 += 32) {
     const int i = i0 + lane;
-    below += __popc(__ballot_sync(0xffffffffu, i < tl.n && tl.base + a.pat_off[p0 + i] < tl.qb * kscale));
+    below += __popc(__ballot_sync(0xffffffffu, i < tl.n && tl.base + a.pat_off[p0 + i] < kb_diag));
   }
   tl.rot = (below < tl.n) ? below : 0;
   return tl;
@@ -167,7 +183,7 @@ struct Cursor {
 
 __device__ __forceinline__ void cursor_seek(const TcArgs& a, Cursor& cu, int T, int G) {
   while (cu.t < T) {
-    const TileList tl = tile_list(a, cu.t, false, a.kscale);
+    const TileList tl = tile_list(a, cu.t, false);
     if (tl.n > 0) {
       cu.n = tl.n;
       cu.base = tl.base;
@@ -214,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
   using L = FwdLayout<D, BK>;
   constexpr int R = L::RING;
-  constexpr int HB = BK / 2;   // key columns per softmax half
+  constexpr int W0 = L::W0;    // key columns of softmax half 0 (half 1: BK - W0)
+  constexpr uint32_t SB = L::SB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   FwdCtrl<R>* c = reinterpret_cast<FwdCtrl<R>*>(smem + L::OFF_CTRL);
@@ -319,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
     const uint32_t sQ = smem_u32(smem + L::OFF_Q);
     const uint32_t sRing = smem_u32(smem + L::OFF_RING);
-    const uint32_t tO = tmem + 256;
+    const uint32_t tO = tmem + 2 * SB;
     uint32_t g = 0, gs = 0, gp = 0;
     int qtiles = 0;   // tiles whose first S was issued
     int otiles = 0;   // tiles whose first PV was issued
@@ -327,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && !(cs.done && cp.done)) {
       const int e = g % R;
       if (take_score(cs, gs, gp)) {
-        const uint32_t tS = tmem + (gs & 1) * 128;
+        const uint32_t tS = tmem + (gs & 1) * SB;
         ok = (cs.j > 0 || mbar_wait(&c->q_full, qtiles & 1, &c->abort, a.spin_ns)) &&
              mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns);
         ok = __all_sync(0xffffffffu, ok);
@@ -351,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++gs;
         cursor_next(a, cs, T, G);
       } else {
-        const uint32_t tP = tmem + (gp & 1) * 128;
+        const uint32_t tP = tmem + (gp & 1) * SB;
         ok = mbar_wait(&c->p_full[gp & 1], (gp >> 1) & 1, &c->abort, a.spin_ns) &&
              mbar_wait(&c->ring_full[e], (g / R) & 1, &c->abort, a.spin_ns) &&
              (cp.j > 0 || mbar_wait(&c->o_free, (otiles & 1) ^ 1, &c->abort, a.spin_ns));
@@ -364,12 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts_k64_w(tO, tP, vd, IDESC_O, cp.j > 0 ? 1u : 0u);
           mma_ts_k64_w(tO, tP + 64, vd + 512, IDESC_O, 1u);
         } else {
-          // half h's keys at P columns [h HB, h HB + HB / 2); 16 keys (8 columns,
-          // 16 V rows = 2048 bytes) per step
+          // 16 keys (8 P columns, 16 V rows = 2048 bytes) per step; the P of
+          // half 0 starts at column 0, that of half 1 at its first score
+          // column W0
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const int hh = kk / (HB / 16), ks = kk % (HB / 16);
-            mma_bf16_ts_w(tO, tP + hh * HB + ks * 8, vd + kk * 128, IDESC_O, (cp.j > 0 || kk > 0) ? 1u : 0u);
+            const int acol = kk < W0 / 16 ? kk * 8 : W0 + (kk - W0 / 16) * 8;
+            mma_bf16_ts_w(tO, tP + acol, vd + kk * 128, IDESC_O, (cp.j > 0 || kk > 0) ? 1u : 0u);
           }
         }
         mma_commit_w(&c->ring_empty[e]);
@@ -391,7 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 8) {
     // ===================== softmax warpgroups =================================
     regs_inc<kSoftmaxRegs>();
+    // One softmax half: HB key columns starting at column c0 of every block
+    // (one instantiation serves both halves when they are equal).
+    auto softmax = [&](auto hb_c) {
+    constexpr int HB = decltype(hb_c)::value;
     const int h = warp >> 2;                  // key-column half of every block
+    const int c0 = h * W0;
     const int w = warp & 3;                   // TMEM lane quarter
     const int row = w * 32 + lane;
     const uint32_t t_row = tmem + (static_cast<uint32_t>(w * 32) << 16);
@@ -415,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return v;
     };
     for (int t = blockIdx.x; ok && t < T; t += G) {
-      const TileList tl = tile_list(a, t, true, TILE / BK);
+      const TileList tl = tile_list(a, t, true);
       const int grow = tl.qb * TILE + row;
       const size_t orow_idx = static_cast<size_t>(tl.bh) * a.Np + grow;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D + h * (D / 2);
@@ -440,18 +463,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, got);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t t_s = t_row + b * 128 + h * HB;   // this half's HB score columns
+        const uint32_t t_s = t_row + b * SB + c0;   // this half's HB score columns
         uint32_t r[HB];
 #pragma unroll
         for (int q4 = 0; q4 < HB / 32; ++q4)
           tmem_ld32(t_s + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
+        if constexpr (HB % 32 == 16) tmem_ld16(t_s + HB / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[HB / 32 * 32]));
         tmem_ld_wait();
         reg_fence(r);
         if (j == j_last && valid_last < BK) {
           // Key columns past the sequence end exist only in the last block.
 #pragma unroll
           for (int i = 0; i < HB; ++i)
-            if (h * HB + i >= valid_last) r[i] = f2u(-INFINITY);
+            if (c0 + i >= valid_last) r[i] = f2u(-INFINITY);
         }
         // p = 2^(s c2 - mref) two columns at a time on the MUFU unit, as
         // bf16 pairs into the first 32 columns of this half's score columns,
@@ -462,12 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t negm = f2pack(-mref, -mref);
           uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
           float mxa = -INFINITY, mxb = -INFINITY;
+          // NP pairs of columns from column e0: bf16 pairs stored from P column e0 / 2
+          auto chunk = [&](auto np_c, int e0, uint32_t (&pk)[decltype(np_c)::value]) {
+            constexpr int NP = decltype(np_c)::value;
 #pragma unroll
-          for (int c16 = 0; c16 < HB / 32; ++c16) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int e = c16 * 32 + 2 * i;
+            for (int i = 0; i < NP; ++i) {
+              const int e = e0 + 2 * i;
               if (track) {
                 if (i & 1) mxb = fmax3(mxb, u2f(r[e]), u2f(r[e + 1]));
                 else mxa = fmax3(mxa, u2f(r[e]), u2f(r[e + 1]));
@@ -481,7 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               f2unpack(pv, pl, ph);
               pk[i] = pack_bf16x2(pl, ph);
             }
+          };
+#pragma unroll
+          for (int c16 = 0; c16 < HB / 32; ++c16) {
+            uint32_t pk[16];
+            chunk(IntC<16>{}, c16 * 32, pk);
             tmem_st16(t_s + c16 * 16, pk);
+          }
+          if constexpr (HB % 32 == 16) {
+            uint32_t pk[8];
+            chunk(IntC<8>{}, HB / 32 * 32, pk);
+            tmem_st8(t_s + HB / 32 * 16, pk);
           }
           mx_out = fmaxf(mxa, mxb);
           float a0, a1, b0, b1;
@@ -540,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q4 = 0; q4 < D / 64; ++q4) {
               uint32_t ro[32];
-              const uint32_t t_o = t_row + 256 + h * (D / 2) + q4 * 32;
+              const uint32_t t_o = t_row + 2 * SB + h * (D / 2) + q4 * 32;
               tmem_ld32(t_o, ro);
               tmem_ld_wait();
               reg_fence(ro);
@@ -584,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q4 = 0; q4 < D / 64; ++q4) {
         uint32_t r[32];
-        tmem_ld32(t_row + 256 + h * (D / 2) + q4 * 32, r);
+        tmem_ld32(t_row + 2 * SB + h * (D / 2) + q4 * 32, r);
         tmem_ld_wait();
         reg_fence(r);
         uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
@@ -607,6 +641,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       c->abort = 1;
       report_status(a.status, CALIBATT_E_TIMEOUT);
     }
+    };
+    if constexpr (2 * W0 == BK) softmax(IntC<W0>{});
+    else if ((warp >> 2) == 0) softmax(IntC<W0>{});
+    else softmax(IntC<BK - W0>{});
   }
 
   tc_fence_before();
@@ -666,13 +704,18 @@ int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcAr
   CUtensorMap tq, tk, tv;
   const uint64_t qrows = static_cast<uint64_t>(a.B) * a.H * a.Np;
   const uint64_t krows = static_cast<uint64_t>(a.B) * a.H * a.Npk;
-  const uint32_t bk = static_cast<uint32_t>(TILE / a.kscale);   // key-block size: 128 or 64
+  const uint32_t bk = static_cast<uint32_t>(a.block_k);
   int rc;
   if ((rc = make_tmap_bf16(&tq, q, qrows, d, TILE)) != CALIBATT_OK) return rc;
   if ((rc = make_tmap_bf16(&tk, k, krows, d, bk)) != CALIBATT_OK) return rc;
   if ((rc = make_tmap_bf16(&tv, v, krows, d, bk)) != CALIBATT_OK) return rc;
-  if (bk == 64) return d == 128 ? launch_fwd<128, 64>(tq, tk, tv, a, s) : launch_fwd<64, 64>(tq, tk, tv, a, s);
-  return d == 128 ? launch_fwd<128, 128>(tq, tk, tv, a, s) : launch_fwd<64, 128>(tq, tk, tv, a, s);
+  switch (bk) {
+    case 64: return d == 128 ? launch_fwd<128, 64>(tq, tk, tv, a, s) : launch_fwd<64, 64>(tq, tk, tv, a, s);
+    case 80: return d == 128 ? launch_fwd<128, 80>(tq, tk, tv, a, s) : launch_fwd<64, 80>(tq, tk, tv, a, s);
+    case 96: return d == 128 ? launch_fwd<128, 96>(tq, tk, tv, a, s) : launch_fwd<64, 96>(tq, tk, tv, a, s);
+    case 144: return d == 128 ? launch_fwd<128, 144>(tq, tk, tv, a, s) : launch_fwd<64, 144>(tq, tk, tv, a, s);
+    default: return d == 128 ? launch_fwd<128, 128>(tq, tk, tv, a, s) : launch_fwd<64, 128>(tq, tk, tv, a, s);
+  }
 }
 
 }  // namespace calibatt

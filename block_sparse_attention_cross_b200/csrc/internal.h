@@ -32,7 +32,7 @@ struct TcArgs {
   const int32_t* pat_ptr;
   const int16_t* pat_off;
   int n_pat, nnz_pat, map_offset;
-  int kscale;              // forward: 128 / key-block size (1 or 2)
+  int block_k;             // forward: key-block size (64, 80, 96, 128 or 144)
   void* o;                 // bf16 [B, H, Np, d]
   float* lse;              // [B, H, Np] natural-log LSE or nullptr
   float* lse2;             // calibration: per-row log2-domain LSE [H * Np]

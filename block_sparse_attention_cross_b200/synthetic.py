@@ -398,3 +398,38 @@ def sweep_masks(w: Workload, layers=40, timesteps=3, seed=1000, lo=0.1, hi=0.6):
                                        block=w.block)[0]
     return out
 
+
+
+def regrid_key_blocks(mask, N, block_k, density, seed, block=128):
+    """The same mask on a grid of ``block_k``-token key blocks (query blocks stay
+    ``block`` tokens): a new key block is kept when it overlaps a kept block of
+    ``mask`` [n_maps, nqb, nkb]; the blocks overlapping the query block's own
+    tokens are always kept; then blocks are dropped (or added) at random to hit
+    round(density * nqb * nkb') exactly, nkb' = ceil(N / block_k).
+    Returns uint8 [n_maps, nqb, nkb'].
+    """
+    rng = np.random.default_rng(seed)
+    n_maps, nqb, nkb = mask.shape
+    nkb2 = -(-N // block_k)
+    lo = np.arange(nkb2) * block_k
+    hi = np.minimum(lo + block_k, N)
+    # coarse block c covers tokens [c block, (c + 1) block): overlap matrix [nkb2, nkb]
+    c_lo = np.arange(nkb) * block
+    over = (lo[:, None] < c_lo[None, :] + block) & (hi[:, None] > c_lo[None, :])
+    q_lo = np.arange(nqb) * block
+    own = (lo[None, :] < q_lo[:, None] + block) & (hi[None, :] > q_lo[:, None])   # [nqb, nkb2]
+    target = int(round(density * nqb * nkb2))
+    out = np.zeros((n_maps, nqb, nkb2), dtype=np.uint8)
+    for m in range(n_maps):
+        keep = ((mask[m] != 0).astype(np.int64) @ over.T.astype(np.int64)) > 0
+        keep |= own
+        cur = int(keep.sum())
+        if cur > target:
+            removable = np.flatnonzero(keep.ravel() & ~own.ravel())
+            drop = rng.choice(removable, size=min(cur - target, removable.size), replace=False)
+            keep.ravel()[drop] = False
+        elif cur < target:
+            free = np.flatnonzero(~keep.ravel())
+            keep.ravel()[rng.choice(free, size=min(target - cur, free.size), replace=False)] = True
+        out[m] = keep
+    return out

@@ -336,3 +336,118 @@ def test_bf16_key_blocks_of_64_wan480_sampled():
     err = np.concatenate(errs)
     assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
     print(f"PARITY wan480 128x64 blocks sampled 16 query blocks max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
+
+
+def run_kv_block_compare(q, k, v, mask, N, d, bk):
+    """Whole-tensor parity with 128-row query blocks and bk-key blocks: the
+    queries are padded to a multiple of 128 and the keys to a multiple of bk
+    (calibatt_sparse_attn_fwd_qk)."""
+    npq, npk = q.shape[2], k.shape[2]
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    v64, vd = bf16_pair(v)
+    bl = cba.compile(torch.from_numpy(mask).cuda(), block_q=128, block_k=bk)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = cba.default_scale(d)
+    o, lse = cba.sparse_attn_fwd_qk(qd, kd, vd, bl, N, N, scale=scale, return_lse=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    H = q.shape[1]
+    O = np.zeros((1, H, npq, d))
+    L = np.full((1, H, npq), -np.inf)
+    for h in range(H):
+        for qb in range(npq // 128):
+            O[0, h, qb * 128:(qb + 1) * 128], L[0, h, qb * 128:(qb + 1) * 128] = oracle.masked_attention_rows(
+                q64, k64, v64, mask, N, 128, bk, scale, 0, h, qb)
+    mx, mn = assert_close(to_np64(o), O, BF16_MAX_ABS, BF16_MEAN_ABS)
+    assert_lse(lse.cpu().numpy(), L, 1e-3)
+    print(f"PARITY bf16 128x{bk} blocks N={N} d={d} max_abs={mx:.3e} mean_abs={mn:.3e}")
+
+
+def _kv_inputs(N, bk, d, H, seed):
+    npq, npk = -(-N // 128) * 128, -(-N // bk) * bk
+    q, _, _ = syn.normal_qkv(1, H, N, npq, d, seed)
+    _, k, v = syn.normal_qkv(1, H, N, npk, d, seed + 1)
+    return q, k, v, npq // 128, npk // bk
+
+
+@pytest.mark.parametrize("bk", [80, 96, 144])
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_key_blocks_80_96_144(bk, d):
+    # Key blocks of the paper page's Table S6 (B_kv = 80, 96, 144 with
+    # B_q = 128): random masks with an empty row, a full row and the padded
+    # last key block kept everywhere; ragged N.
+    N, H = 1900, 3
+    q, k, v, nqb, nkb = _kv_inputs(N, bk, d, H, 71)
+    rng = np.random.default_rng(72)
+    mask = (rng.random((H, nqb, nkb)) < 0.4).astype(np.uint8)
+    mask[0, 4, :] = 0
+    mask[1, 7, :] = 1
+    mask[2, :, nkb - 1] = 1
+    run_kv_block_compare(q, k, v, mask, N, d, bk)
+
+
+@pytest.mark.parametrize("bk,N", [(144, 934), (80, 1000), (96, 1086)])
+def test_bf16_key_blocks_last_block_mostly_padding(bk, N):
+    # The last key block holds fewer real keys than the first softmax half's
+    # columns (so the second half of that block is all padding), and it is
+    # the first block some query tiles walk.
+    d, H = 128, 2
+    q, k, v, nqb, nkb = _kv_inputs(N, bk, d, H, 81)
+    rng = np.random.default_rng(82)
+    mask = (rng.random((H, nqb, nkb)) < 0.3).astype(np.uint8)
+    mask[:, nqb - 1, :] = 0
+    mask[:, nqb - 1, nkb - 1] = 1          # only the padded last block
+    mask[0, 0, nkb - 1] = 1
+    run_kv_block_compare(q, k, v, mask, N, d, bk)
+
+
+def test_bf16_key_blocks_80_large_score_jumps():
+    # The redo / O-rescale paths with unequal halves (48 + 32 columns).
+    N, H, d, bk = 1900, 2, 128, 80
+    q, k, v, nqb, nkb = _kv_inputs(N, bk, d, H, 91)
+    rng = np.random.default_rng(92)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    q = (q + 8.0 * u).astype(np.float32)
+    g = 12.0 * np.repeat(rng.permutation(k.shape[2] // 16 + 1), 16)[:k.shape[2]]
+    k = (k + g[None, None, :, None] * u).astype(np.float32)
+    mask = (rng.random((H, nqb, nkb)) < 0.5).astype(np.uint8)
+    mask[0, 5, :] = 1
+    run_kv_block_compare(q, k, v, mask, N, d, bk)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bk", [80, 96, 144])
+def test_bf16_key_blocks_wan480_sampled(bk):
+    # The Wan 480p call with the key grid of Table S6 at its reported sparsity
+    # (the 128 x 128 structured mask regridded to bk-key blocks).
+    w = syn.WORKLOADS["wan480_25"]
+    dens = {80: 0.354, 96: 0.359, 144: 0.369}[bk]
+    mask = syn.regrid_key_blocks(syn.workload_mask(w, density=dens), w.N, bk, dens, 17)
+    q, k, v = syn.video_qkv(w)
+    npk = mask.shape[2] * bk
+    kp = np.zeros((1, w.H, npk, w.d), np.float32)
+    vp = np.zeros_like(kp)
+    kp[:, :, :w.N] = k[:, :, :w.N]
+    vp[:, :, :w.N] = v[:, :, :w.N]
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(kp)
+    v64, vd = bf16_pair(vp)
+    del q, k, v, kp, vp
+    bl = cba.compile(torch.from_numpy(mask).cuda(), block_q=128, block_k=bk)
+    scale = cba.default_scale(w.d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = cba.sparse_attn_fwd_qk(qd, kd, vd, bl, w.N, w.N, scale=scale, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    rng = np.random.default_rng(18)
+    errs = []
+    for h, qb in [(0, 0), (w.H - 1, w.nqb - 1)] + [(int(rng.integers(w.H)), int(rng.integers(w.nqb)))
+                                                   for _ in range(10)]:
+        O, _ = oracle.masked_attention_rows(q64, k64, v64, mask, w.N, 128, bk, scale, 0, h, qb)
+        errs.append(np.abs(to_np64(o[0, h, qb * 128:(qb + 1) * 128]) - O).ravel())
+    err = np.concatenate(errs)
+    assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
+    print(f"PARITY wan480 128x{bk} blocks (density {mask.mean():.3f}) sampled 12 query blocks "
+          f"max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
