@@ -144,12 +144,18 @@ def test_calibrate_wan_config_full_size_against_float64_oracle():
     keeps = [oracle.select_topk(E, 0.25) for E in Eo]
     m64, _, _ = oracle.vote(np.stack(keeps), oracle.min_votes_for(0.5, I), Eo)
     tie = np.zeros((len(heads), w.nqb), bool)
+    close = np.zeros((len(heads), w.nqb), bool)
     for E in Eo:
         tie |= near_tie_rows(E, k)
+        # rows whose k-th and (k+1)-th energies are closer than twice the
+        # measured GPU energy error: the only rows whose selection the
+        # float32 energies can change
+        srt = -np.sort(-E, axis=-1)
+        close |= (srt[..., k - 1] - srt[..., k]) < 2 * err.max()
     diff_rows = (mask_g != m64).any(axis=-1)
-    print(f"PARITY calibrate wan480 end to end: rows_differing={int(diff_rows.sum())} "
-          f"near_tie_rows={int(tie.sum())} of {tie.size}")
-    assert not (diff_rows & ~tie).any()
+    print(f"PARITY calibrate wan480 end to end: rows_differing={int(diff_rows.sum())} of {tie.size}; rows within "
+          f"2x the energy error of a tie={int(close.sum())}; near-tie rows by the 1e-4 relative rule={int(tie.sum())}")
+    assert not (diff_rows & ~close).any()
 
 
 @pytest.mark.slow
