@@ -25,8 +25,9 @@ configurations, each timed on the device and checked against the float64
 oracle on a sample: the Wan 720p and Mochi calls (20% kept), the sweep of
 120 calls (40 layers x 3 timesteps x 40 heads), one calibration pass of 8
 Wan 480p inputs, the Wan 480p call with each key-block size of the paper
-page's Table S6 (64 ... 144 keys) at its reported sparsity, and the tiny
-fp32 case.
+page's Table S6 (64 ... 144 keys) at its reported sparsity, the
+spatial-repetition path at Table S4's anchor counts with the
+spatial-similarity score of one input, and the tiny fp32 case.
 
 ``--gpus N`` without a launcher starts N replica processes itself (one per
 GPU, the torchrun environment set for each); under torchrun the world size
@@ -596,6 +597,61 @@ def _key_block_workload(device, pk):
     return rec
 
 
+def _spatial_workload(device):
+    """The spatial-repetition path at the paper page's Table S4 setting (Wan 480p, 40 heads, k of 30 spatial
+    rows per frame, every key) and the spatial-similarity score of one input (Figure 6(a), Figure S13)."""
+    import torch
+    import block_sparse_attention_cross_b200 as cba
+    import oracle
+    w = workload(None, "wan480_25")
+    g = w.grid
+    (q, k, v), host = _qkv_device(w, device)
+    scale = cba.default_scale(w.d)
+    rec = {"anchor_rows": {}}
+    base_ms = None
+    for ka in (30, 15, 10, 5, 4, 3):
+        plan = cba.anchor_plan(g.frames, g.rows, g.cols, ka, w.Np, device)
+        bl = cba.compile(torch.ones((w.H, plan.npq // 128, w.Np // 128), dtype=torch.uint8, device=device))
+        o = None
+
+        def call():
+            nonlocal o
+            o = cba.anchor_attention(q, k, v, plan, bl=bl)
+
+        tot, _ = time_calls(call, 10, 3, torch)
+        ms = tot / 10
+        base_ms = ms if ka == 30 else base_ms
+        ent = {"row_sparsity": round(1 - ka / g.rows, 4), "ms_per_call": round(ms, 3),
+               "speedup_vs_all_rows": round(base_ms / ms, 3)}
+        if ka == 5:
+            call()
+            torch.cuda.synchronize()
+            errs = []
+            for h, qb in ((3, 17), (31, 200)):
+                toks = list(range(qb * 128, (qb + 1) * 128))
+                want = oracle.anchor_attention_tokens(host[0], host[1], host[2], w.N, g.frames, g.rows, g.cols, ka,
+                                                      scale, 0, h, toks)
+                errs.append(np.abs(o[0, h, toks[0]:toks[-1] + 1].float().cpu().numpy().astype(np.float64) - want))
+            ent["parity_sampled"] = dict(_parity(errs), blocks=2)
+        rec["anchor_rows"][f"k={ka}"] = ent
+    s = None
+
+    def sim():
+        nonlocal s
+        s = cba.spatial_similarity(q[0], k[0], w.N, g.frames, g.rows, g.cols)
+
+    tot, _ = time_calls(sim, 3, 1, torch)
+    sim()
+    torch.cuda.synchronize()
+    want = oracle.spatial_similarity(host[0][0, 5:6], host[1][0, 5:6], w.N, g.frames, g.rows, g.cols, scale)
+    flops = 6.0 * w.N * w.N * w.d * w.H   # STATS pass (2 N^2 d) + the pair pass (4 N^2 d), per head
+    rec["spatial_similarity"] = {"ms_per_input": round(tot / 3, 2), "qk_tflops": round(flops / (tot / 3 / 1e3) / 1e12, 1),
+                                 "score_head5": float(s[5].item()),
+                                 "abs_err_vs_float64_head5": float(abs(float(s[5].item()) - want[0])),
+                                 "bound": 1e-4}
+    return rec
+
+
 def other_workloads(device, pk):
     """The configurations besides the headline call, each timed and sampled against the oracle (N = 1)."""
     import torch
@@ -605,6 +661,7 @@ def other_workloads(device, pk):
                      ("sweep_4800_maps", lambda: _sweep_workload(device, pk)),
                      ("calibration_8_inputs", lambda: _calibration_workload(device)),
                      ("key_blocks_table_s6", lambda: _key_block_workload(device, pk)),
+                     ("spatial_repetition", lambda: _spatial_workload(device)),
                      ("tiny_fp32", lambda: _tiny_fp32_workload(device))):
         t0 = time.perf_counter()
         rec[name] = fn()

@@ -71,14 +71,17 @@ def launch_count():
 
 
 def min_votes_for(rho, n_inputs):
-    """Integer agreement threshold: keep a block iff votes / I >= rho."""
-    v = math.ceil(round(float(rho) * int(n_inputs), 9))
-    return int(min(max(v, 0), int(n_inputs)))
+    """Integer agreement threshold: keep a block iff votes / I >= rho (``calibatt_min_votes``)."""
+    out = ctypes.c_int32(0)
+    check(load().calibatt_min_votes(float(rho), int(n_inputs), ctypes.byref(out)))
+    return out.value
 
 
 def topk_count(frac, nkb):
-    """Kept key blocks per row in top-k mode: ceil(frac * nkb) clamped to [1, nkb]."""
-    return int(min(nkb, max(1, math.ceil(frac * nkb))))
+    """Kept key blocks per row in top-k mode: ceil(frac * nkb) clamped to [1, nkb] (``calibatt_topk_count``)."""
+    out = ctypes.c_int32(0)
+    check(load().calibatt_topk_count(float(frac), int(nkb), ctypes.byref(out)))
+    return out.value
 
 
 @dataclass
@@ -125,11 +128,16 @@ class BlockList:
         return self.nnz / float(self.n_maps * self.n_q_blocks * self.n_k_blocks)
 
     def kept_blocks(self, map_offset=0, n=None):
-        """Kept blocks of maps [map_offset, map_offset + n): computed on the GPU from the pattern pool."""
+        """Kept blocks of maps [map_offset, map_offset + n) (``calibatt_blocklist_kept``; synchronizes)."""
         n = self.n_maps - map_offset if n is None else n
-        r0, r1 = map_offset * self.n_q_blocks, (map_offset + n) * self.n_q_blocks
-        lens = self.pat_ptr[1:] - self.pat_ptr[:-1]
-        return int(lens[self.row_pat[r0:r1].long()].sum().item())
+        dev = self.row_pat.device
+        ws = torch.empty(1, dtype=torch.int64, device=dev)
+        out = ctypes.c_int64(0)
+        s = self.as_struct()
+        with torch.cuda.device(dev):
+            check(load().calibatt_blocklist_kept(ctypes.byref(s), int(map_offset), int(n), ctypes.byref(out), _ptr(ws),
+                                                 8, _stream(dev)))
+        return out.value
 
 
 def sparse_attn_fwd(q, k, v, bl: BlockList, N, scale=None, map_offset=0, return_lse=False, out=None, lse=None,

@@ -78,6 +78,9 @@ EXPORTS = {
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "calibatt_blocklist_bytes": (c_int, [c_int, c_int, c_int64, c_int32, c_int32, POINTER(c_int64),
                                          POINTER(c_int64)]),
+    "calibatt_min_votes": (c_int, [c_double, c_int, POINTER(c_int32)]),
+    "calibatt_topk_count": (c_int, [c_double, c_int, POINTER(c_int32)]),
+    "calibatt_blocklist_kept": (c_int, [c_void_p, c_int, c_int, POINTER(c_int64), c_void_p, c_size_t, c_void_p]),
     "calibatt_spatial_similarity_workspace_size": (c_int, [c_int, c_int, POINTER(c_size_t)]),
     "calibatt_spatial_similarity": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                             c_int, c_float, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),

@@ -122,6 +122,26 @@ __global__ void k_skiplist_widths(const int32_t* __restrict__ counts, int rows_p
   }
 }
 
+// Sum of the pattern lengths of rows [r0, r1): the kept blocks of those rows.
+__global__ void k_rows_kept(const int32_t* __restrict__ row_pat, const int32_t* __restrict__ pat_ptr, long long r0,
+                            long long r1, unsigned long long* out) {
+  __shared__ unsigned long long part[8];
+  unsigned long long acc = 0;
+  for (long long r = r0 + static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; r < r1;
+       r += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int p = row_pat[r];
+    acc += static_cast<unsigned long long>(pat_ptr[p + 1] - pat_ptr[p]);
+  }
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
+    atomicAdd(out, t);
+  }
+}
+
 constexpr int kMaxPcts = 64;
 constexpr int kMaxSkipKeyBlocks = 16384;   // histogram of <= 8193 bins in shared memory
 
@@ -241,6 +261,29 @@ int calibatt_skiplist_sizes(const int32_t* counts, int n_maps, int nqb, int nkb,
   return CALIBATT_OK;
 }
 
+int calibatt_min_votes(double rho, int n_inputs, int32_t* min_votes) {
+  if (min_votes == nullptr) return set_error(CALIBATT_E_INVALID, "min_votes is NULL");
+  if (n_inputs <= 0 || !std::isfinite(rho)) return set_error(CALIBATT_E_INVALID, "bad rho or input count");
+  // ceil(rho I), after rounding rho I to 9 decimals so that a product such as
+  // 0.3 * 10 = 3.0000000000000004 counts as 3
+  const double v = std::nearbyint(rho * n_inputs * 1e9) / 1e9;
+  double c = std::ceil(v);
+  if (c < 0) c = 0;
+  if (c > n_inputs) c = n_inputs;
+  *min_votes = static_cast<int32_t>(c);
+  return CALIBATT_OK;
+}
+
+int calibatt_topk_count(double frac, int nkb, int32_t* k) {
+  if (k == nullptr) return set_error(CALIBATT_E_INVALID, "k is NULL");
+  if (nkb <= 0 || !(frac > 0.0) || frac > 1.0) return set_error(CALIBATT_E_INVALID, "need 0 < frac <= 1, nkb > 0");
+  double v = std::ceil(frac * nkb);
+  if (v < 1) v = 1;
+  if (v > nkb) v = nkb;
+  *k = static_cast<int32_t>(v);
+  return CALIBATT_OK;
+}
+
 int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, int32_t nnz_pat, int64_t* csr_bytes,
                              int64_t* pool_bytes) {
   if (csr_bytes == nullptr || pool_bytes == nullptr) return set_error(CALIBATT_E_INVALID, "NULL outputs");
@@ -248,6 +291,33 @@ int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, in
   const long long rows = static_cast<long long>(n_maps) * nqb;
   *csr_bytes = (rows + 1) * 8 + nnz * 2;                             // int64 row_ptr + int16 col
   *pool_bytes = rows * 8 + (static_cast<long long>(n_pat) + 1) * 4 + static_cast<long long>(nnz_pat) * 2;
+  return CALIBATT_OK;
+}
+
+int calibatt_blocklist_kept(const calibatt_blocklist* bl, int map_offset, int n_maps, int64_t* kept, void* workspace,
+                            size_t workspace_bytes, calibatt_stream_t stream) {
+  if (bl == nullptr || kept == nullptr || bl->row_pat == nullptr || bl->pat_ptr == nullptr)
+    return set_error(CALIBATT_E_INVALID, "NULL argument");
+  if (map_offset < 0 || n_maps <= 0 || static_cast<long long>(map_offset) + n_maps > bl->n_maps)
+    return set_error(CALIBATT_E_INVALID, "maps [%d, %d) outside the list's %d maps", map_offset, map_offset + n_maps,
+                     bl->n_maps);
+  if (workspace == nullptr || workspace_bytes < 8) return set_error(CALIBATT_E_WORKSPACE, "need 8 bytes of workspace");
+  if (reinterpret_cast<uintptr_t>(workspace) & 7u) return set_error(CALIBATT_E_INVALID, "workspace must be 8-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned long long* d = static_cast<unsigned long long*>(workspace);
+  int rc;
+  if ((rc = cuda_ok(cudaMemsetAsync(d, 0, 8, s), "cudaMemsetAsync"))) return rc;
+  const long long r0 = static_cast<long long>(map_offset) * bl->n_q_blocks;
+  const long long r1 = r0 + static_cast<long long>(n_maps) * bl->n_q_blocks;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>((r1 - r0 + 255) / 256, 148ll * 4));
+  k_rows_kept<<<grid, 256, 0, s>>>(bl->row_pat, bl->pat_ptr, r0, r1, d);
+  count_launch();
+  if ((rc = check_launch("k_rows_kept"))) return rc;
+  unsigned long long h = 0;
+  if ((rc = cuda_ok(cudaMemcpyAsync(&h, d, 8, cudaMemcpyDeviceToHost, s), "cudaMemcpyAsync")) ||
+      (rc = cuda_ok(cudaStreamSynchronize(s), "cudaStreamSynchronize")))
+    return rc;
+  *kept = static_cast<int64_t>(h);
   return CALIBATT_OK;
 }
 

@@ -509,6 +509,32 @@ int calibatt_skiplist_sizes(const int32_t* counts, int n_maps, int nqb, int nkb,
 int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, int32_t nnz_pat, int64_t* csr_bytes,
                              int64_t* pool_bytes);
 
+/*
+ * calibatt_min_votes -- the integer agreement threshold of the vote (paper
+ * page, Figure 3(b) and Figure 7: a block is kept when at least a fraction rho
+ * of the calibration inputs keep it): min_votes = ceil(rho n_inputs), with
+ * rho n_inputs rounded to 9 decimals first (so 0.3 * 10 gives 3), clamped to
+ * [0, n_inputs].  Host arithmetic only.
+ */
+int calibatt_min_votes(double rho, int n_inputs, int32_t* min_votes);
+
+/*
+ * calibatt_topk_count -- key blocks kept per query-block row by the top-k
+ * selection (paper page, Figure 5(a)): ceil(frac nkb) clamped to [1, nkb], the
+ * count calibatt_select_vote uses.  Host arithmetic only; frac in (0, 1].
+ */
+int calibatt_topk_count(double frac, int nkb, int32_t* k);
+
+/*
+ * calibatt_blocklist_kept -- the number of kept blocks of maps [map_offset,
+ * map_offset + n_maps) of a compiled block list (the sum of their rows'
+ * pattern lengths), for per-call density and FLOP counts.  workspace: 8 bytes
+ * of device memory (8-byte aligned).  Synchronizes `stream`.
+ */
+int calibatt_blocklist_kept(const calibatt_blocklist* bl, int map_offset, int n_maps, int64_t* kept, void* workspace,
+                            size_t workspace_bytes, calibatt_stream_t stream);
+
+
 
 /*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the

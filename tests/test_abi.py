@@ -200,3 +200,19 @@ def test_gathered_query_forward_and_gather_validation(lib):
     assert lib.calibatt_gather_rows(None, fake, fake, 1, 4, 4, 256, None) == _lib.E_INVALID
     assert lib.calibatt_gather_rows(fake, fake, fake, 1, 4, 4, 200, None) == _lib.E_INVALID     # not a multiple of 16
     assert lib.calibatt_gather_rows(ctypes.c_void_p(0x10008), fake, fake, 1, 4, 4, 256, None) == _lib.E_INVALID
+
+
+def test_integer_parameters_match_the_oracle(lib):
+    # calibatt_min_votes / calibatt_topk_count are host arithmetic in the
+    # library: the same integers as the oracle's definitions over a grid.
+    import oracle
+    import block_sparse_attention_cross_b200 as cba
+    for n in (1, 2, 3, 5, 8, 10, 16, 33):
+        for rho in (0.0, 0.1, 0.25, 0.3, 1 / 3, 0.5, 0.6, 0.7, 0.875, 0.9, 1.0):
+            assert cba.min_votes_for(rho, n) == oracle.min_votes_for(rho, n), (rho, n)
+    for nkb in (1, 7, 256, 350, 591):
+        for frac in (1e-9, 0.1, 0.2, 0.25, 1 / 3, 0.5, 0.999, 1.0):
+            assert cba.topk_count(frac, nkb) == oracle.topk_count(frac, nkb), (frac, nkb)
+    out = ctypes.c_int32(0)
+    assert lib.calibatt_topk_count(0.0, 10, ctypes.byref(out)) == _lib.E_INVALID
+    assert lib.calibatt_min_votes(float("nan"), 4, ctypes.byref(out)) == _lib.E_INVALID

@@ -61,3 +61,32 @@ def test_sweep_maps_full_size():
     want = oracle.compile_blocklist(masks)
     for key in ("row_base", "row_pat", "pat_ptr", "pat_off", "csr_row_ptr", "csr_col"):
         assert np.array_equal(got[key], want[key]), key
+
+
+def test_blocklist_kept_counts_match_the_masks():
+    # calibatt_blocklist_kept: kept blocks of any map range, from the pattern pool.
+    rng = np.random.default_rng(44)
+    masks = (rng.random((9, 11, 23)) < rng.random((9, 1, 1))).astype(np.uint8)
+    masks[3] = 0
+    bl = cba.compile(torch.from_numpy(masks).cuda())
+    for mo, n in ((0, 9), (0, 1), (3, 1), (2, 5), (8, 1)):
+        assert bl.kept_blocks(mo, n) == int(masks[mo:mo + n].sum())
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs a second visible GPU")
+def test_forward_and_energy_on_a_second_device_after_the_first():
+    # Launch set-up (shared-memory limits, SM counts) is per device: the same
+    # process runs the kernels on device 0, then on device 1.
+    from block_sparse_attention_cross_b200 import synthetic as syn
+    H, N, Np, d = 2, 1000, 1024, 128
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 5)
+    mask = np.ones((H, 8, 8), np.uint8)
+    outs = []
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            t = [torch.from_numpy(x).to(f"cuda:{dev}").to(torch.bfloat16) for x in (q, k, v)]
+            bl = cba.compile(torch.from_numpy(mask).to(f"cuda:{dev}"))
+            outs.append(cba.sparse_attn_fwd(*t, bl, N).cpu())
+            E = cba.block_energy(t[0][0], t[1][0], N)
+            assert torch.allclose(E[:, :, :].sum(-1), torch.ones_like(E[:, :, 0]), atol=1e-4)
+    assert torch.equal(outs[0], outs[1])
