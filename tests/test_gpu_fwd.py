@@ -451,3 +451,82 @@ def test_bf16_key_blocks_wan480_sampled(bk):
     assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
     print(f"PARITY wan480 128x{bk} blocks (density {mask.mean():.3f}) sampled 12 query blocks "
           f"max_abs={err.max():.3e} mean_abs={err.mean():.3e}")
+
+
+@pytest.mark.parametrize("N", [1, 129])
+def test_bf16_degenerate_lengths(N):
+    # One real token (the row attends to itself only: O = v_0, LSE = s_00) and
+    # a last block holding a single real token; padding rows come back 0 / -inf.
+    d, H = 128, 2
+    Np = -(-N // 128) * 128
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 101)
+    nb = Np // 128
+    mask = np.ones((H, nb, nb), np.uint8)
+    run_full_compare(q, k, v, mask, N, 128, "bf16", d)
+
+
+@pytest.mark.slow
+def test_bf16_longest_rows_2048_key_blocks():
+    # The longest supported list: 2 048 key blocks per row (262 144 tokens,
+    # one head), a ragged end, 1% of the blocks plus the diagonal kept;
+    # sampled whole query blocks against the oracle.
+    H, d, nb = 1, 128, 2048
+    N, Np = nb * 128 - 5, nb * 128
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 103)
+    rng = np.random.default_rng(104)
+    mask = (rng.random((H, nb, nb)) < 0.01).astype(np.uint8)
+    mask[0, np.arange(nb), np.arange(nb)] = 1
+    mask[0, :, nb - 1] = 1
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    v64, vd = bf16_pair(v)
+    bl = cba.compile(torch.from_numpy(mask).cuda())
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    scale = cba.default_scale(d)
+    o, lse = cba.sparse_attn_fwd(qd, kd, vd, bl, N, scale=scale, return_lse=True, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    errs = []
+    for qb in (0, 1, 1000, nb - 1):
+        O, L = oracle.masked_attention_rows(q64, k64, v64, mask, N, 128, 128, scale, 0, 0, qb)
+        rows = slice(qb * 128, (qb + 1) * 128)
+        errs.append(np.abs(to_np64(o[0, 0, rows]) - O).ravel())
+        assert_lse(lse[0, 0, rows].cpu().numpy(), L, 1e-3)
+    err = np.concatenate(errs)
+    assert err.max() <= BF16_MAX_ABS and err.mean() <= BF16_MEAN_ABS, (err.max(), err.mean())
+    print(f"PARITY bf16 2048 key blocks per row (N={N}) sampled 4 query blocks max_abs={err.max():.3e} "
+          f"mean_abs={err.mean():.3e}")
+
+
+def test_bf16_forward_replays_in_a_cuda_graph():
+    # The forward enqueues only kernels on the caller's stream (descriptors are
+    # encoded on the host, nothing is allocated), so a sequence of calls can be
+    # captured once and replayed; replays give the eager results bit for bit.
+    H, N, Np, d = 3, 2000, 2048, 128
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 111)
+    rng = np.random.default_rng(112)
+    masks = (rng.random((3 * H, 16, 16)) < 0.4).astype(np.uint8)
+    masks[:, np.arange(16), np.arange(16)] = 1
+    _, qd = bf16_pair(q)
+    _, kd = bf16_pair(k)
+    _, vd = bf16_pair(v)
+    bl = cba.compile(torch.from_numpy(masks).cuda())
+    eager = [cba.sparse_attn_fwd(qd, kd, vd, bl, N, map_offset=mo) for mo in (0, H, 2 * H)]
+    outs = [torch.empty_like(qd) for _ in range(3)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):   # warm-up on the capture stream
+        for mo, o in zip((0, H, 2 * H), outs):
+            cba.sparse_attn_fwd(qd, kd, vd, bl, N, map_offset=mo, out=o)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for mo, o in zip((0, H, 2 * H), outs):
+            cba.sparse_attn_fwd(qd, kd, vd, bl, N, map_offset=mo, out=o)
+    for _ in range(2):
+        for o in outs:
+            o.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for e, o in zip(eager, outs):
+            assert torch.equal(e, o)
