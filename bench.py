@@ -418,8 +418,12 @@ def _parity(errs):
             "within_bound": bool(e.max() <= 2e-2 and e.mean() <= 2e-3)}
 
 
-def _sampled_fwd_errors(w, host, mask, picks, scale, gpu_out):
-    _, _, outs = run_oracle_sample(w, host, mask, picks, scale, keep_outputs=True)
+def _sampled_fwd_errors(w, host, mask, picks, scale, gpu_out, timing=None):
+    t, kept, outs = run_oracle_sample(w, host, mask, picks, scale, keep_outputs=True)
+    if timing is not None:
+        timing.update({"value": kept_flops(kept, w.d, 1) / t / 1e12, "unit": UNIT, "cores": cpu_threads(),
+                       "kind": "oracle", "sample": f"{len(picks)} (head, query-block) pairs ({kept} kept blocks), "
+                                                   f"float64 numpy, extrapolated in kept blocks; {t:.2f} s"})
     return [np.abs(gpu_out[0, h, qb * w.block:(qb + 1) * w.block].float().cpu().numpy().astype(np.float64) - o)
             for (h, qb), o in zip(picks, outs)]
 
@@ -442,8 +446,9 @@ def _fwd_workload(name, device, pk):
     cba.sparse_attn_fwd(q, k, v, bl, w.N, out=out)
     torch.cuda.synchronize()
     kept = kept_flops(bl.nnz, w.d, w.B) / (ms / 1e3) / 1e12
-    picks = sampled_blocks(w, 4, 3)
-    errs = _sampled_fwd_errors(w, host, mask_np, picks, cba.default_scale(w.d), out)
+    picks = sampled_blocks(w, 4, 8)
+    cpu = {}
+    errs = _sampled_fwd_errors(w, host, mask_np, picks, cba.default_scale(w.d), out, timing=cpu)
     g = w.grid
     return {"shape": f"{g.frames}x{g.rows}x{g.cols}" + (f" + {g.text_tokens} text" if g.text_tokens else "") +
                      f" = {w.N} tokens (padded {w.Np}), {w.H} heads, d={w.d}, bf16, 128x128 blocks",
@@ -451,7 +456,7 @@ def _fwd_workload(name, device, pk):
             "frac_of_bf16_burst": round(kept / pk["bf16_burst"], 4),
             "dense_equiv_tflops": round(4.0 * w.N * w.N * w.d * w.H * w.B / (ms / 1e3) / 1e12, 2),
             "full_mask_ms": round(tf / 5, 4), "speedup_vs_full_mask": round(tf / 5 / ms, 3),
-            "parity_sampled": dict(_parity(errs), blocks=len(picks))}
+            "parity_sampled": dict(_parity(errs), blocks=len(picks)), "cpu_baseline": cpu}
 
 
 def _sweep_workload(device, pk):
