@@ -76,7 +76,7 @@ constexpr uint32_t kTmemCols = 512;
 // and O stay far below the fp32 range for |v| < 2^47.
 constexpr float kRescaleThreshold = 64.0f;
 
-// D: head dim; BK: key-block size (128 or 64; query blocks are always 128).
+// D: head dim; BK: key-block size (64, 80, 96, 128 or 144; query blocks are always 128).
 template <int D, int BK>
 struct FwdLayout {
   static constexpr uint32_t QBOX_BYTES = TILE * 64 * 2;  // 128 rows x 64 bf16 (one 128-byte swizzle span)

@@ -125,15 +125,18 @@ uint64_t calibatt_get_spin_limit_ns(void);
  *  q, k, v  [B, H, Np, d] of `dtype` (16-byte aligned); o the same shape
  *           and type (written); lse [B, H, Np] float32 or NULL.
  *  scale    the softmax scale (normally the float32 of 1/sqrt(d)).
- *  bl       host pointer to a compiled block list with block_q = block_k
- *           and n_q_blocks = n_k_blocks = Np / block_q;
- *           map_offset + H <= bl->n_maps.  The mask is shared by the batch.
+ *  bl       host pointer to a compiled block list with n_q_blocks =
+ *           Np / block_q and n_k_blocks = Np / block_k (Np a multiple of
+ *           both, Np - N below either); map_offset + H <= bl->n_maps.  The
+ *           mask is shared by the batch.  Key blocks that do not divide the
+ *           query padding use calibatt_sparse_attn_fwd_qk.
  *  dev_status optional device int32 (see conventions).
  * Supported: CALIBATT_BF16 with d in {64, 128}, block_q = 128 and block_k
- * in {128, 64} (tcgen05 tensor cores, fp32 accumulation, P rounded to bf16
- * for the PV product; paper page, Table S6 compares key-block sizes);
- * CALIBATT_FP32 with d in {64, 128}, block in {64, 128} (FFMA).  Anything
- * else returns CALIBATT_E_UNSUPPORTED.
+ * in {64, 80, 96, 128, 144} (tcgen05 tensor cores, fp32 accumulation, P
+ * rounded to bf16 for the PV product; paper page, Table S6 compares these
+ * key-block sizes); CALIBATT_FP32 with d in {64, 128}, block_q = block_k in
+ * {64, 128} (FFMA).  At most 2048 key blocks per row.  Anything else returns
+ * CALIBATT_E_UNSUPPORTED.
  */
 int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int H, int N, int Np, int d, int dtype, float scale,
