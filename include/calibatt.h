@@ -134,9 +134,9 @@ uint64_t calibatt_get_spin_limit_ns(void);
  * Supported: CALIBATT_BF16 with d in {64, 128}, block_q = 128 and block_k
  * in {64, 80, 96, 128, 144} (tcgen05 tensor cores, fp32 accumulation, P
  * rounded to bf16 for the PV product; paper page, Table S6 compares these
- * key-block sizes); CALIBATT_FP32 with d in {64, 128}, block_q = block_k in
- * {64, 128} (FFMA).  At most 2048 key blocks per row.  Anything else returns
- * CALIBATT_E_UNSUPPORTED.
+ * key-block sizes); CALIBATT_FP32 with d in {64, 128}, block_q and block_k
+ * in {64, 128} (FFMA).  At most 2048 key blocks per row.  Anything else
+ * returns CALIBATT_E_UNSUPPORTED.
  */
 int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int H, int N, int Np, int d, int dtype, float scale,
