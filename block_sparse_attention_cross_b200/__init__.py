@@ -365,7 +365,7 @@ def block_energy(q, k, N, block_q=128, block_k=128, scale=None, status=None, wor
     _need_cuda(q, k)
     H, Np, d = q.shape
     scale = default_scale(d) if scale is None else float(scale)
-    E = torch.empty((H, Np // block_q, Np // block_k), device=q.device, dtype=torch.float32)
+    E = torch.empty((H, Np // block_q, -(-int(N) // block_k)), device=q.device, dtype=torch.float32)
     ws = _calib_workspace(H, N, Np, d, block_q, block_k, q.device) if workspace is None else workspace
     with torch.cuda.device(q.device):
         check(load().calibatt_block_energy(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q, block_k,
@@ -385,7 +385,7 @@ def block_energy_noalloc(q, k, N, block_q=128, block_k=128, scale=None, status=N
     _need_cuda(q, k)
     H, Np, d = q.shape
     scale = default_scale(d) if scale is None else float(scale)
-    E = torch.empty((H, Np // block_q, Np // block_k), device=q.device, dtype=torch.float32) if out is None else out
+    E = torch.empty((H, Np // block_q, -(-int(N) // block_k)), device=q.device, dtype=torch.float32) if out is None else out
     _need_cuda(E, status)
     with torch.cuda.device(q.device):
         check(load().calibatt_block_energy_noalloc(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q,
@@ -428,7 +428,7 @@ def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mo
     _need_cuda(*q_list, *k_list)
     H, Np, d = q_list[0].shape
     dev = q_list[0].device
-    nqb, nkb = Np // block_q, Np // block_k
+    nqb, nkb = Np // block_q, -(-int(N) // block_k)
     scale = default_scale(d) if scale is None else float(scale)
     if votes is None:
         votes = torch.zeros((H, nqb, nkb), dtype=torch.int32, device=dev)

@@ -356,9 +356,9 @@ int calibatt_sparse_attn_fwd_streamed(const void* q_host, const void* k_host, co
 
 int calibatt_calibrate_workspace_size(int H, int N, int Np, int d, int block_q, int block_k, size_t* bytes) {
   if (bytes == nullptr) return set_error(CALIBATT_E_INVALID, "bytes is NULL");
-  if (H <= 0 || N <= 0 || Np < N || d <= 0 || block_q <= 0 || block_k <= 0 || Np % block_q || Np % block_k)
+  if (H <= 0 || N <= 0 || Np < N || d <= 0 || block_q <= 0 || block_k <= 0 || Np % block_q)
     return set_error(CALIBATT_E_INVALID, "bad sizes");
-  const size_t nqb = Np / block_q, nkb = Np / block_k;
+  const size_t nqb = Np / block_q, nkb = (static_cast<size_t>(N) + block_k - 1) / block_k;
   // per-row LSE [H*Np] + energies [H*nqb*nkb], each 256-byte aligned
   *bytes = ((static_cast<size_t>(H) * Np * 4 + 255) & ~size_t(255)) + ((H * nqb * nkb * 4 + 255) & ~size_t(255)) + 256;
   return CALIBATT_OK;
@@ -370,10 +370,11 @@ namespace calibatt {
 
 int energy_impl(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int block_q, int block_k,
                 float scale, float* energy_out, float* lse_ws, int32_t* dev_status, cudaStream_t s) {
-  const int nqb = Np / block_q, nkb = Np / block_k;
+  const int nqb = Np / block_q, nkb = (N + block_k - 1) / block_k;
   if (dtype == CALIBATT_BF16) {
     TcArgs a{};
-    a.B = 1; a.H = H; a.N = N; a.Np = Np; a.nqb = nqb; a.nkb = nkb;
+    // nkb: 128-key tiles walked; the energies use nke blocks of block_k keys
+    a.B = 1; a.H = H; a.N = N; a.Np = Np; a.nqb = nqb; a.nkb = Np / 128; a.block_k = block_k; a.nke = nkb;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.lse2 = lse_ws; a.energy = energy_out; a.status = dev_status; a.spin_ns = spin_limit_ns();
     return launch_tc_energy(q, k, d, a, s);
@@ -387,22 +388,27 @@ int energy_impl(const void* q, const void* k, int H, int N, int Np, int d, int d
 int check_energy_args(const void* q, const void* k, int H, int N, int Np, int d, int dtype, int block_q,
                       int block_k, float scale) {
   if (q == nullptr || k == nullptr) return set_error(CALIBATT_E_INVALID, "q and k must be non-NULL");
-  if (H <= 0 || N <= 0 || Np < N || d <= 0 || block_q <= 0 || block_k <= 0 || Np % block_q || Np % block_k)
+  if (H <= 0 || N <= 0 || Np < N || d <= 0 || block_q <= 0 || block_k <= 0 || Np % block_q)
     return set_error(CALIBATT_E_INVALID, "bad sizes H=%d N=%d Np=%d d=%d", H, N, Np, d);
-  if ((Np - N) >= block_k || (Np - N) >= block_q)
-    return set_error(CALIBATT_E_INVALID, "Np - N must be smaller than one block");
+  if ((Np - N) >= block_q) return set_error(CALIBATT_E_INVALID, "Np - N must be smaller than one query block");
   if (!(scale > 0.f) || !std::isfinite(scale)) return set_error(CALIBATT_E_INVALID, "scale must be finite and > 0");
   if (!aligned16(q) || !aligned16(k)) return set_error(CALIBATT_E_INVALID, "q and k must be 16-byte aligned");
   if (static_cast<long long>(H) * Np >= (1ll << 31)) return set_error(CALIBATT_E_UNSUPPORTED, "H*Np too large");
   if (dtype == CALIBATT_BF16) {
-    if (!(d == 64 || d == 128) || block_q != 128 || block_k != 128)
-      return set_error(CALIBATT_E_UNSUPPORTED, "bf16 energies support d in {64,128} with 128x128 blocks");
-    if (Np / block_k > 1024) return set_error(CALIBATT_E_UNSUPPORTED, "at most 1024 key blocks");
+    if (!(d == 64 || d == 128) || block_q != 128 ||
+        !(block_k == 64 || block_k == 80 || block_k == 96 || block_k == 128 || block_k == 144))
+      return set_error(CALIBATT_E_UNSUPPORTED,
+                       "bf16 energies support d in {64,128}, 128-row query blocks and key blocks of 64, 80, 96, 128 or "
+                       "144");
+    if (Np / 128 > 2048 || (N + block_k - 1) / block_k > 2048)
+      return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks");
     return CALIBATT_OK;
   }
   if (dtype == CALIBATT_FP32) {
     if (!(d == 64 || d == 128) || !(block_q == 64 || block_q == 128) || !(block_k == 64 || block_k == 128))
       return set_error(CALIBATT_E_UNSUPPORTED, "fp32 energies support d in {64,128}, blocks in {64,128}");
+    if (Np % block_k || (Np - N) >= block_k)
+      return set_error(CALIBATT_E_INVALID, "fp32 energies need Np a multiple of block_k and Np - N below it");
     return CALIBATT_OK;
   }
   return set_error(CALIBATT_E_UNSUPPORTED, "unknown dtype %d", dtype);
@@ -490,7 +496,7 @@ int calibatt_calibrate(const void* const* q_list, const void* const* k_list, int
   int rc;
   for (int n = 0; n < n_inputs; ++n)
     if ((rc = check_energy_args(q_list[n], k_list[n], H, N, Np, d, dtype, block_q, block_k, scale))) return rc;
-  const int nqb = Np / block_q, nkb = Np / block_k;
+  const int nqb = Np / block_q, nkb = (N + block_k - 1) / block_k;
   if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
   if (select_mode == CALIBATT_SELECT_TOPK) {
     if (!(select_param > 0.0) || select_param > 1.0) return set_error(CALIBATT_E_INVALID, "top-k fraction must be in (0,1]");

@@ -6,7 +6,10 @@
 // STATS computes each query row's dense log-sum-exp (log2 domain) over all
 // real keys; ENERGY recomputes the scores, sums exp2(s - LSE) inside every key
 // block and reduces the 128 rows of the query block in a fixed order, so the
-// result is deterministic.
+// result is deterministic.  Scores are always produced in 128-key tiles; for a
+// key-block size BK other than 128 (Table S6: 64, 80, 96, 144) a tile covers up
+// to three key blocks, whose boundaries fall on 16-column chunks, so every
+// chunk's sum goes to exactly one block.
 //
 // CTA = one 128-row query tile of one head, 8 warps:
 //   warp 0      TMA producer: the Q tile once, then every K tile into a
@@ -34,7 +37,7 @@ constexpr int TILE = 128;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kRing = 4;
-constexpr int kMaxBlocks = 1024;  // key blocks per row (partials buffer)
+constexpr int kMaxBlocks = 2048;  // key blocks per row (partials buffer)
 
 template <int D>
 struct EnergyLayout {
@@ -169,6 +172,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(w * 32) << 16);
     const float c2 = a.scale_log2;
     float* part = reinterpret_cast<float*>(smem + L::OFF_PART);
+    const int bk = a.block_k;
+    if (MODE == MODE_ENERGY && bk != TILE) {
+      // Each warp owns the slots part[4 * kb + w]; they accumulate across tiles.
+      for (int kb = lane; kb < a.nke; kb += 32) part[4 * kb + w] = 0.f;
+      __syncwarp();
+    }
     const float lse2_row =
         (MODE == MODE_ENERGY && grow < a.N) ? a.lse2[static_cast<size_t>(h) * a.Np + grow] : 0.f;
     float m = -INFINITY;
@@ -199,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < TILE; ++i)
           if (i >= valid) s[i] = -INFINITY;
       }
-      if (MODE == MODE_ENERGY) {
+      if (MODE == MODE_ENERGY && bk == TILE) {
         float rs = 0.f;
         if (grow < a.N) {
 #pragma unroll
@@ -208,6 +217,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
         if (lane == 0) part[j * 4 + w] = rs;
+      } else if (MODE == MODE_ENERGY) {
+        // Key blocks kb0, kb0+1, kb0+2 meet this tile at columns [0,b1),
+        // [b1,b2), [b2,128); b1 and b2 are multiples of 16.
+        const int kb0 = (j * TILE) / bk;
+        const int b1 = (kb0 + 1) * bk - j * TILE;
+        const int b2 = b1 + bk;
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f;
+        if (grow < a.N) {
+#pragma unroll
+          for (int c = 0; c < TILE / 16; ++c) {
+            float cs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cs += ex2_approx(fmaf(s[c * 16 + i], c2, -lse2_row));
+            if (c * 16 < b1) r0 += cs;
+            else if (c * 16 < b2) r1 += cs;
+            else r2 += cs;
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          r0 += __shfl_xor_sync(0xffffffffu, r0, o);
+          r1 += __shfl_xor_sync(0xffffffffu, r1, o);
+          r2 += __shfl_xor_sync(0xffffffffu, r2, o);
+        }
+        if (lane == 0) {
+          part[4 * kb0 + w] += r0;
+          if (b1 < TILE && kb0 + 1 < a.nke) part[4 * (kb0 + 1) + w] += r1;
+          if (b2 < TILE && kb0 + 2 < a.nke) part[4 * (kb0 + 2) + w] += r2;
+        }
+        __syncwarp();
       } else {
         float mx = s[0];
 #pragma unroll
@@ -231,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         const int rows = min(TILE, a.N - qb * TILE);
         const float inv_rows = 1.f / static_cast<float>(rows);
-        float* erow = a.energy + (static_cast<size_t>(h) * a.nqb + qb) * a.nkb;
-        for (int j = row; j < n; j += TILE) {
+        const int ne = (bk == TILE) ? n : a.nke;
+        float* erow = a.energy + (static_cast<size_t>(h) * a.nqb + qb) * ne;
+        for (int j = row; j < ne; j += TILE) {
           const float tot = ((part[4 * j + 0] + part[4 * j + 1]) + part[4 * j + 2]) + part[4 * j + 3];
           erow[j] = tot * inv_rows;
         }

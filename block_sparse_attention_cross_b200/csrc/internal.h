@@ -32,7 +32,8 @@ struct TcArgs {
   const int32_t* pat_ptr;
   const int16_t* pat_off;
   int n_pat, nnz_pat, map_offset;
-  int block_k;             // forward: key-block size (64, 80, 96, 128 or 144)
+  int block_k;             // key-block size (64, 80, 96, 128 or 144)
+  int nke;                 // energies: key blocks of block_k keys, ceil(N / block_k)
   void* o;                 // bf16 [B, H, Np, d]
   float* lse;              // [B, H, Np] natural-log LSE or nullptr
   float* lse2;             // calibration: per-row log2-domain LSE [H * Np]

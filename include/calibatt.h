@@ -298,11 +298,20 @@ int calibatt_repetition_flags(const float* scores, int n_inputs, int n_maps, flo
  * Table S5 ("block energies"):
  *     E[h, qb, kb] = (1 / #rows(qb)) sum_{i in qb, i < N} sum_{j in kb, j < N} softmax_j(scale q_i.k_j)
  * with the softmax over ALL keys j < N (dense, unmasked).  Every row of E
- * sums to 1.
- *  q, k       [H, Np, d] of `dtype`;  energy_out [H, Np/block_q, Np/block_k] float32.
+ * sums to 1.  The key grid covers the real keys: nkb = ceil(N / block_k)
+ * blocks, the last one partial when block_k does not divide N.
+ *  q, k       [H, Np, d] of `dtype`, Np a multiple of block_q, Np - N < block_q;
+ *  energy_out [H, Np/block_q, ceil(N/block_k)] float32 (written).
  *  workspace  >= calibatt_calibrate_workspace_size bytes (256-byte aligned).
- * Supported: CALIBATT_BF16 with d in {64,128}, blocks 128 (tensor cores);
- * CALIBATT_FP32 with d in {64,128}, blocks in {64,128} (FFMA).
+ * Supported: CALIBATT_BF16 with d in {64,128}, block_q = 128 and block_k in
+ * {64, 80, 96, 128, 144} (the key-block sizes of Table S6), at most 2 048
+ * query blocks and 2 048 key blocks (tensor cores);
+ * CALIBATT_FP32 with d in {64,128}, block_q and block_k in {64,128}, Np also
+ * a multiple of block_k with Np - N < block_k (FFMA).
+ * Errors: CALIBATT_E_INVALID (NULL, sizes, scale), CALIBATT_E_UNSUPPORTED
+ * (shape outside the list), CALIBATT_E_WORKSPACE (workspace too small).
+ * Asynchronous; dev_status (may be NULL) receives CALIBATT_E_TIMEOUT if a
+ * bounded wait in the kernel expired.
  */
 int calibatt_block_energy(const void* q, const void* k, int H, int N, int Np, int d, int dtype,
                           int block_q, int block_k, float scale, float* energy_out,
@@ -349,6 +358,8 @@ int calibatt_finalize_mask(const int32_t* votes, const float* energy_sum, int H,
  * the counts simply add up).  If mask_out != NULL, finishes with
  * calibatt_finalize_mask(min_votes).
  *  q_list, k_list  HOST arrays of n_inputs device pointers, each [H, Np, d].
+ *  votes_inout, energy_sum_inout, mask_out  [H, Np/block_q, ceil(N/block_k)].
+ * Shapes as calibatt_block_energy.
  */
 int calibatt_calibrate(const void* const* q_list, const void* const* k_list, int n_inputs,
                        int H, int N, int Np, int d, int dtype, int block_q, int block_k,

@@ -53,13 +53,15 @@ def block_energy(q, k, N, block_q, block_k, scale):
     """Block energies of one calibration input.
 
     ``q, k``: [H, Np, d] (any float dtype, read exactly).  Returns
-    E [H, nqb, nkb] float64.  Padded query rows (>= N) are excluded from the
-    mean; padded keys (>= N) take no probability mass.
+    E [H, nqb, nkb] float64 with nkb = ceil(N / block_k): the key grid covers
+    the real keys only (Table S6 varies the key-block size independently of
+    the query block, and a key block past the sequence would hold no key).
+    Padded query rows (>= N) are excluded from the mean.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     H, Np, d = q.shape
-    nqb, nkb = Np // block_q, Np // block_k
+    nqb, nkb = Np // block_q, -(-N // block_k)
     scale = float(np.float64(scale))
     E = np.zeros((H, nqb, nkb))
     for h in range(H):
@@ -75,8 +77,7 @@ def block_energy(q, k, N, block_q, block_k, scale):
 
 def block_energy_row(q, k, N, block_q, block_k, scale, h, qb):
     """One row E[h, qb, :] of ``block_energy`` (for sampled checks at full size)."""
-    Np = np.shape(q)[1]
-    nkb = Np // block_k
+    nkb = -(-N // block_k)
     r0, r1 = qb * block_q, min(qb * block_q + block_q, N)
     if r1 <= r0:
         return np.zeros(nkb)

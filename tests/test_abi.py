@@ -125,6 +125,9 @@ def test_workspace_queries(lib):
     assert lib.calibatt_calibrate_workspace_size(40, 32760, 32768, 128, 128, 128, ctypes.byref(n)) == _lib.OK
     assert n.value >= 40 * 32768 * 4 + 40 * 256 * 256 * 4
     assert lib.calibatt_calibrate_workspace_size(40, 32760, 32760, 128, 128, 128, ctypes.byref(n)) == _lib.E_INVALID
+    # key blocks of 80 over 32 760 real keys: ceil(32760 / 80) = 410 blocks per row
+    assert lib.calibatt_calibrate_workspace_size(40, 32760, 32768, 128, 128, 80, ctypes.byref(n)) == _lib.OK
+    assert n.value >= 40 * 32768 * 4 + 40 * 256 * 410 * 4
     assert lib.calibatt_compile_workspace_size(4800, 256, 256, ctypes.byref(n)) == _lib.OK
     assert n.value > 4800 * 256 * 8
     assert lib.calibatt_compile_workspace_size(0, 256, 256, ctypes.byref(n)) == _lib.E_INVALID
@@ -136,6 +139,15 @@ def test_calibration_and_compile_validation(lib):
                                      None, None) == _lib.E_UNSUPPORTED
     assert lib.calibatt_block_energy(fake, fake, 2, 1000, 1024, 128, _lib.BF16, 128, 128, 0.1, fake, fake, 16,
                                      None, None) == _lib.E_WORKSPACE
+    # Table S6 key blocks pass validation (then fail on the workspace); others are unsupported
+    for bk in (64, 80, 96, 144):
+        assert lib.calibatt_block_energy(fake, fake, 2, 1000, 1024, 128, _lib.BF16, 128, bk, 0.1, fake, fake, 16,
+                                         None, None) == _lib.E_WORKSPACE
+    assert lib.calibatt_block_energy(fake, fake, 2, 1000, 1024, 128, _lib.BF16, 128, 112, 0.1, fake, fake, 1 << 30,
+                                     None, None) == _lib.E_UNSUPPORTED
+    # 2 048 query tiles of 128 rows with 64-key blocks: 4 096 key blocks per row, above the limit
+    assert lib.calibatt_block_energy(fake, fake, 1, 262144, 262144, 64, _lib.BF16, 128, 64, 0.1, fake, fake,
+                                     1 << 30, None, None) == _lib.E_UNSUPPORTED
     assert lib.calibatt_select_vote(fake, 2, 8, 8, 5, 0.1, fake, fake, None) == _lib.E_INVALID
     assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_TOPK, 0.0, fake, fake, None) == _lib.E_INVALID
     assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_ENERGY, 1.0, fake, fake, None) == _lib.E_INVALID

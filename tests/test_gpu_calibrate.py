@@ -48,6 +48,77 @@ def test_block_energy(dtype, d, block):
     np.testing.assert_allclose(E[:, :nreal].sum(axis=-1), 1.0, atol=1e-4)
 
 
+@pytest.mark.parametrize("d,bk", [(128, 64), (128, 80), (128, 96), (128, 144), (64, 80), (64, 144)])
+def test_block_energy_key_block_sizes(d, bk):
+    # Table S6 key grids (B_kv = 64, 80, 96, 144 against 128-row query
+    # blocks): a 128-key score tile meets up to three key blocks; ragged N,
+    # so the last key block is partial.
+    H = 2
+    w, inputs = small_inputs(1, H, syn.VideoGrid(2, 20, 51), d, seed_base=30)
+    q, k = inputs[0]
+    q64, qd = bf16_pair(q)
+    k64, kd = bf16_pair(k)
+    scale = cba.default_scale(d)
+    E = cba.block_energy(qd, kd, w.N, 128, bk, scale=scale).cpu().numpy().astype(np.float64)
+    nke = -(-w.N // bk)
+    assert E.shape == (H, w.Np // 128, nke)
+    Eo = oracle.block_energy(q64, k64, w.N, 128, bk, scale)
+    err = np.abs(E - Eo).max()
+    print(f"PARITY energy bf16 d={d} 128x{bk} blocks N={w.N} max_abs={err:.3e}")
+    assert err <= 5e-5, err
+    nreal = -(-w.N // 128)
+    np.testing.assert_allclose(E[:, :nreal].sum(axis=-1), 1.0, atol=1e-4)
+
+
+def test_calibrate_key_blocks_of_80_drive_the_forward():
+    # The Table S6 pipeline at B_kv = 80: calibrate on 80-key blocks, compile,
+    # run the forward with keys padded to a multiple of 80.  Discrete stages
+    # are bit-exact on the GPU's energies; the forward matches the oracle.
+    H, I, bk, d = 2, 3, 80, 128
+    w, inputs = small_inputs(I, H, syn.VideoGrid(3, 30, 52), d, seed_base=40)
+    pairs = [(bf16_pair(q), bf16_pair(k)) for q, k in inputs]
+    qd = [p[0][1] for p in pairs]
+    kd = [p[1][1] for p in pairs]
+    mv = cba.min_votes_for(0.5, I)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mask, votes, esum = cba.calibrate(qd, kd, w.N, block_k=bk, select_param=0.3, rho=0.5, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    nke = -(-w.N // bk)
+    assert mask.shape == (H, w.Np // 128, nke)
+    Eg = [cba.block_energy(q, k, w.N, 128, bk).cpu().numpy() for q, k in zip(qd, kd)]
+    keeps = [oracle.select_topk(E, 0.3) for E in Eg]
+    m_o, v_o, e_o = oracle.vote(np.stack(keeps), mv, np.stack(Eg))
+    assert np.array_equal(votes.cpu().numpy(), v_o)
+    assert np.array_equal(esum.cpu().numpy(), e_o)
+    assert np.array_equal(mask.cpu().numpy(), m_o)
+    # forward on input 0 with the calibrated 80-key mask
+    npk = nke * bk
+    q64, k64 = pairs[0][0][0], pairs[0][1][0]
+    rng = np.random.default_rng(41)
+    v32 = rng.standard_normal((H, npk, d)).astype(np.float32)
+    v32[:, w.N:] = 0.0
+    v64, vd = bf16_pair(v32)
+    kk = np.zeros((H, npk, d))
+    kk[:, :w.N] = k64[:, :w.N]
+    kd80 = torch.zeros((1, H, npk, d), dtype=torch.bfloat16, device="cuda")
+    kd80[0, :, :w.N] = kd[0][:, :w.N]
+    bl = cba.compile(mask, block_q=128, block_k=bk)
+    o = cba.sparse_attn_fwd_qk(qd[0][None], kd80, vd[None], bl, w.N, w.N, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    m = mask.cpu().numpy()
+    scale = cba.default_scale(d)
+    err = 0.0
+    for h, qb in ((0, 0), (0, 7), (1, 3), (1, w.Np // 128 - 1)):
+        ref, _ = oracle.masked_attention_rows(q64[None], kk[None], v64[None], m, w.N, 128, bk, scale, 0, h, qb)
+        got = o[0, h, qb * 128:(qb + 1) * 128].float().cpu().numpy()
+        real = min(128, w.N - qb * 128)
+        err = max(err, np.abs(got[:real] - ref[:real]).max())
+    print(f"PARITY calibrate+forward 128x{bk} blocks max_abs={err:.3e}")
+    assert err <= 2e-2, err
+
+
 def test_select_vote_finalize_bit_exact():
     rng = np.random.default_rng(4)
     H, nqb, nkb, I = 3, 9, 37, 5
