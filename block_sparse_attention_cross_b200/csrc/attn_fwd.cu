@@ -6,13 +6,21 @@
 // kept-block list; only the kept K/V tiles are loaded (TMA) and multiplied
 // (tcgen05), so a skipped block costs neither bytes nor FLOPs.
 //
-// Templated on the head dim D (128 or 64) and the key-block size BK (64, 80,
-// 96, 128 or 144; query blocks are always 128 rows; the paper page's Table S6
-// compares these key-block sizes).  The text below describes BK = 128.  In
-// general the two softmax halves take W0 = BK / 2 rounded up to a multiple of
-// 16 key columns and BK - W0 (80 = 48 + 32, 144 = 80 + 64), so that each
-// half's probabilities feed whole PV K steps of 16 keys; score buffers are 128
-// TMEM columns apart (160 for BK = 144) and O follows them.
+// Two kernels, both templated on the head dim D (128 or 64) and the
+// key-block size BK (64, 80, 96, 128 or 144; query blocks are always 128
+// rows; the paper page's Table S6 compares these key-block sizes):
+//   k_attn_fwd_pp  two query tiles per CTA, one thread per query row (see
+//                  the section that defines it); used wherever its two tiles'
+//                  scores and accumulators fit in TMEM: every shape but
+//                  D = 128 with 144-key blocks.
+//   k_attn_fwd     one query tile per CTA, each block's keys split between
+//                  two warps of the same rows (described here); used for
+//                  D = 128 with 144-key blocks.
+// The text below describes k_attn_fwd at BK = 128.  In general its two
+// softmax halves take W0 = BK / 2 rounded up to a multiple of 16 key columns
+// and BK - W0 (80 = 48 + 32, 144 = 80 + 64), so that each half's
+// probabilities feed whole PV K steps of 16 keys; score buffers are 128 TMEM
+// columns apart (160 for BK = 144) and O follows them.
 //
 // Persistent CTA (one per SM, one query tile at a time), 12 warps:
 //   warps 0-3   softmax, key columns 0-63 of each block (warp w: rows 32w..32w+31)
@@ -115,6 +123,7 @@ struct FwdCtrl {
 
 template <int V>
 using IntC = std::integral_constant<int, V>;
+
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
@@ -653,14 +662,489 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ===========================================================================
+// Two query tiles per CTA ("slots" 0 and 1), one thread per query row.
+//
+// Each slot has its own softmax warpgroup (warps 0-3: slot 0, warps 4-7:
+// slot 1; warp w's rows are TMEM lanes 32 (w % 4) ...), its own Q buffer,
+// score buffer S_s, accumulator O_s, TMA producer (warps 8 and 11) and K/V
+// ring; warp 9 issues every MMA, warp 10 is idle.  A thread holds its row's
+// whole block of scores in registers, so the row maximum needs no exchange
+// between warps: the block maximum is taken first and the exponentials use
+// the reference that follows from it.  The two warps that share an SM
+// sub-partition belong to different slots; the tensor core alternates
+// between the slots (PV_0, S_0, PV_1, S_1, ...), so while one slot's scores
+// are being computed the other slot's warps exponentiate, and one slot's
+// TMEM loads, stores and waits overlap the other slot's exponentials.
+//
+// TMEM (512 columns): slot s owns [256 s, 256 s + 256): S_s at
+// [256 s, 256 s + BK) and O_s at [256 s + OC, 256 s + OC + D) with OC = 128
+// (160 for BK = 144).  P overwrites the first BK / 2 columns of S_s as bf16
+// pairs: the A operand of the PV MMA.  With one score buffer per slot the
+// order per slot is S(j), softmax(j), PV(j), S(j + 1): S(j + 1) may overwrite
+// P(j) because the in-order tensor pipe has consumed it, and the commit that
+// signals S(j + 1) also covers PV(j), so O_s can be rescaled as soon as the
+// scores of block j + 1 are visible.
+// ===========================================================================
+
+template <int D, int BK>
+struct PpLayout {
+  static constexpr uint32_t QBOX_BYTES = TILE * 64 * 2;
+  static constexpr uint32_t KBOX_BYTES = BK * 64 * 2;
+  static constexpr uint32_t Q_BYTES = TILE * D * 2;
+  static constexpr uint32_t KV_BYTES = BK * D * 2;
+  static constexpr uint32_t OC = BK <= 128 ? 128 : 160;   // O_s column offset inside the slot
+  static_assert(BK % 16 == 0 && BK >= 64 && OC + D <= 256 && BK <= OC, "key-block size / head dim");
+  static_assert(KV_BYTES % 1024 == 0 && KBOX_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned tiles");
+  static constexpr uint32_t OFF_Q = 0;   // Q tiles of slots 0 and 1
+  static constexpr uint32_t OFF_RING = 2 * Q_BYTES;
+  static constexpr uint32_t CTRL_BYTES = 1024;
+  static constexpr uint32_t BUDGET = 232448 - OFF_RING - CTRL_BYTES - 1024;
+  // K/V tiles per slot ring (each slot's producer fills its own ring)
+  static constexpr int RING = (BUDGET / (2 * KV_BYTES)) > 4 ? 4 : static_cast<int>(BUDGET / (2 * KV_BYTES));
+  static_assert(RING >= 2, "ring");
+  static constexpr uint32_t OFF_CTRL = OFF_RING + 2 * RING * KV_BYTES;
+  static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
+};
+
+template <int RING>
+struct PpCtrl {
+  uint64_t ring_full[2][RING], ring_empty[2][RING];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full[2], o_free[2];
+  uint64_t drain[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void pp_cursor_init(const TcArgs& a, Cursor& cu, int slot, int T, int G) {
+  cu.t = blockIdx.x + slot * G;
+  cu.done = false;
+  cursor_seek(a, cu, T, 2 * G);
+}
+
+constexpr int kPpProducer0 = 8, kPpMma = 9, kPpProducer1 = 11;   // warp 10 idle
+
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_attn_fwd_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const TcArgs a) {
+  using L = PpLayout<D, BK>;
+  constexpr int R = L::RING;
+  constexpr uint32_t OC = L::OC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  PpCtrl<R>* c = reinterpret_cast<PpCtrl<R>*>(smem + L::OFF_CTRL);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int G = gridDim.x;
+  const int T = a.B * a.H * a.nqb;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      for (int e = 0; e < R; ++e) {
+        mbar_init(&c->ring_full[s][e], 1);
+        mbar_init(&c->ring_empty[s][e], 1);
+      }
+      mbar_init(&c->q_full[s], 1);
+      mbar_init(&c->q_empty[s], 1);
+      mbar_init(&c->s_full[s], 1);
+      mbar_init(&c->p_full[s], 128);
+      mbar_init(&c->o_full[s], 1);
+      mbar_init(&c->o_free[s], 128);
+      mbar_init(&c->drain[s], 1);
+    }
+    c->abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == kPpMma) {
+    tmem_alloc(&c->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c->tmem_base;
+
+  if (warp >= 8) regs_dec<kControlRegs>();
+  if (warp == kPpProducer0 || warp == kPpProducer1) {
+    // ===================== TMA producer of one slot ===========================
+    // Per kept block of the slot's walk: its K tile, then its V tile, into
+    // the slot's own ring (the order the slot's MMA warp consumes them).
+    const int s = warp == kPpProducer1;
+    Cursor cu;
+    pp_cursor_init(a, cu, s, T, G);
+    uint32_t g = 0;   // ring fills
+    int qf = 0;
+    bool ok = true;
+    const uint64_t pol = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
+    uint8_t* ring = smem + L::OFF_RING + s * R * L::KV_BYTES;
+    while (ok && !cu.done) {
+      if (cu.j == 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty[s], (qf & 1) ^ 1, &c->abort, a.spin_ns));
+        if (!ok) break;
+        mbar_arrive_expect_tx_w(&c->q_full[s], L::Q_BYTES);
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_2d_w(smem + L::OFF_Q + s * L::Q_BYTES + x * L::QBOX_BYTES, &tmQ, x * 64,
+                        cu.bh * a.Np + cu.qb * TILE, &c->q_full[s], pol_q);
+        ++qf;
+      }
+      const int row = cu.bh * a.Npk + cursor_kb(a, cu) * BK;
+#pragma unroll 1
+      for (int kv = 0; kv < 2; ++kv) {
+        const int e = g % R;
+        ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[s][e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
+        if (!ok) break;
+        mbar_arrive_expect_tx_w(&c->ring_full[s][e], L::KV_BYTES);
+        const CUtensorMap* tm = kv ? &tmV : &tmK;
+#pragma unroll
+        for (int x = 0; x < D / 64; ++x)
+          tma_load_2d_w(ring + e * L::KV_BYTES + x * L::KBOX_BYTES, tm, x * 64, row, &c->ring_full[s][e], pol);
+        ++g;
+      }
+      cursor_next(a, cu, T, 2 * G);
+    }
+    if (lane == 0) {
+      if (!ok) {
+        c->abort = 1;
+        report_status(a.status, CALIBATT_E_TIMEOUT);
+      }
+      // Drain: every copy issued must have landed before the CTA may exit.
+      for (int e = 0; e < R; ++e) {
+        const uint32_t fills = (g > static_cast<uint32_t>(e)) ? (g - 1 - e) / R + 1 : 0;
+        if (fills > 0) mbar_wait(&c->ring_full[s][e], (fills - 1) & 1, nullptr, a.spin_ns);
+      }
+      if (qf > 0) mbar_wait(&c->q_full[s], (qf - 1) & 1, nullptr, a.spin_ns);
+    }
+  } else if (warp == kPpMma) {
+    // ===================== MMA issuer =========================================
+    // Per kept block b of a slot's walk: S(b), then (once the slot's softmax
+    // has stored P(b)) PV(b) followed by S(b + 1).  The slots are served in
+    // turn.  Both slots start together, but the second slot's next scores
+    // queue behind the first slot's PV and S, so from the second block on the
+    // slots run half a period apart: one slot exponentiates while the other
+    // slot's products run, and each slot's MMA wait is another's softmax.
+    // (Measured: serving the slot whose P arrives first, polling both
+    // barriers, was slower; so were PV(b) and S(b + 1) issued as one burst
+    // and P signalled in two key halves.)
+    Cursor cu0, cu1;
+    pp_cursor_init(a, cu0, 0, T, G);
+    pp_cursor_init(a, cu1, 1, T, G);
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, BK, false);
+    constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
+    uint32_t g0 = 0, g1 = 0;     // ring tiles consumed per slot
+    uint32_t gb0 = 0, gb1 = 0;   // blocks whose PV was issued per slot
+    int qt0 = 0, qt1 = 0;        // tiles whose first S was issued per slot
+    int ot0 = 0, ot1 = 0;        // tiles whose first PV was issued per slot
+    bool ok = true;
+    // The slot is a compile-time constant in both steps, so every slot's
+    // state stays in registers.
+    auto issue_s = [&](auto s_c) {
+      constexpr int s = decltype(s_c)::value;
+      Cursor& cu = s ? cu1 : cu0;
+      uint32_t& g = s ? g1 : g0;
+      int& qt = s ? qt1 : qt0;
+      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::KV_BYTES);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::Q_BYTES);
+      const uint32_t tS = tmem + s * 256;
+      const int e = g % R;
+      bool w = (cu.j > 0 || mbar_wait(&c->q_full[s], qt & 1, &c->abort, a.spin_ns)) &&
+               mbar_wait(&c->ring_full[s][e], (g / R) & 1, &c->abort, a.spin_ns);
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      const uint32_t sK = sRing + e * L::KV_BYTES;
+      if (D == 128 && BK == TILE) {
+        mma_ss_k128_w(tS, sdesc_sw128(sQ, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::QBOX_BYTES >> 4);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32, 16, 1024);
+          mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      }
+      mma_commit_w(&c->s_full[s]);
+      mma_commit_w(&c->ring_empty[s][e]);
+      if (cu.j == 0) ++qt;
+      if (cu.j == cu.n - 1) mma_commit_w(&c->q_empty[s]);
+      ++g;
+      return true;
+    };
+    // PV(b) of slot s (its P is stored), then the slot's next S.
+    auto issue_pv = [&](auto s_c) {
+      constexpr int s = decltype(s_c)::value;
+      Cursor& cu = s ? cu1 : cu0;
+      uint32_t& g = s ? g1 : g0;
+      uint32_t& gb = s ? gb1 : gb0;
+      int& ot = s ? ot1 : ot0;
+      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::KV_BYTES);
+      const uint32_t tS = tmem + s * 256;
+      const uint32_t tO = tS + OC;
+      const int e = g % R;
+      bool w = mbar_wait(&c->ring_full[s][e], (g / R) & 1, &c->abort, a.spin_ns) &&
+               (cu.j > 0 || mbar_wait(&c->o_free[s], (ot & 1) ^ 1, &c->abort, a.spin_ns));
+      if (!__all_sync(0xffffffffu, w)) return false;
+      tc_fence_after();
+      // P: BK / 2 columns of bf16 pairs at the start of S_s; 16 keys (8
+      // columns, 16 V rows = 2048 bytes) per K step.
+      const uint64_t vd = sdesc_sw128(sRing + e * L::KV_BYTES, L::KBOX_BYTES, 1024);
+      if (BK == TILE) {
+        mma_ts_k128_w(tO, tS, vd, IDESC_O, cu.j > 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_bf16_ts_w(tO, tS + kk * 8, vd + kk * 128, IDESC_O, (cu.j > 0 || kk > 0) ? 1u : 0u);
+      }
+      mma_commit_w(&c->ring_empty[s][e]);
+      if (cu.j == 0) ++ot;
+      if (cu.j == cu.n - 1) mma_commit_w(&c->o_full[s]);
+      ++g;
+      ++gb;
+      cursor_next(a, cu, T, 2 * G);
+      return cu.done ? true : issue_s(s_c);
+    };
+    bool due0 = false, due1 = false;   // an S was issued whose PV is outstanding
+    if (!cu0.done) ok = due0 = issue_s(IntC<0>{});
+    if (ok && !cu1.done) ok = due1 = issue_s(IntC<1>{});
+    int turn = 0;
+    while (ok && (due0 || due1)) {
+      // the slots in turn (suspending waits)
+      const int s = (due0 && (turn == 0 || !due1)) ? 0 : 1;
+      const bool w = mbar_wait(&c->p_full[s], (s ? gb1 : gb0) & 1, &c->abort, a.spin_ns);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+      if (s == 0) {
+        ok = issue_pv(IntC<0>{});
+        due0 = !cu0.done;
+      } else {
+        ok = issue_pv(IntC<1>{});
+        due1 = !cu1.done;
+      }
+      turn = s ^ 1;
+    }
+    if (!ok && lane == 0) {
+      c->abort = 1;
+      report_status(a.status, CALIBATT_E_TIMEOUT);
+    }
+    __syncwarp();
+    mma_commit_w(&c->drain[0]);
+    mbar_wait(&c->drain[0], 0, nullptr, a.spin_ns);
+  } else if (warp < 8) {
+    // ===================== softmax warpgroups =================================
+    regs_inc<kSoftmaxRegs>();
+    const int slot = warp >> 2;
+    const int w = warp & 3;                   // TMEM lane quarter
+    const int row = w * 32 + lane;
+    const uint32_t t_s = tmem + (static_cast<uint32_t>(w * 32) << 16) + slot * 256;   // this row of S_slot
+    const uint32_t t_o = t_s + OC;                                                      // and of O_slot
+    const float c2 = a.scale_log2;
+    const uint64_t c2x2 = f2pack(c2, c2);
+    uint32_t gb = 0;   // blocks of non-empty tiles consumed by this slot
+    int tiles = 0;     // non-empty tiles finished
+    bool ok = true;
+    for (int t = blockIdx.x + slot * G; ok && t < T; t += 2 * G) {
+      const TileList tl = tile_list(a, t, true);
+      const int grow = tl.qb * TILE + row;
+      const size_t orow_idx = static_cast<size_t>(tl.bh) * a.Np + grow;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + orow_idx * D;
+      if (tl.n == 0) {
+        uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = z;
+        if (a.lse != nullptr) a.lse[orow_idx] = -INFINITY;
+        continue;
+      }
+      const int kb_last = tl.base + a.pat_off[tl.p0 + tl.n - 1];
+      const int valid_last = (kb_last == a.nkb - 1) ? (a.Nk - kb_last * BK) : BK;
+      const int j_last = (tl.n - 1 - tl.rot + tl.n) % tl.n;   // walk position of the highest kept block
+      float m = -INFINITY;
+      float l = 0.f;
+      float s_best = -INFINITY;   // largest raw score of the row (normalisation fix-up)
+      for (int j = 0; j < tl.n; ++j, ++gb) {
+        const bool got = mbar_wait(&c->s_full[slot], gb & 1, &c->abort, a.spin_ns);
+        ok = __all_sync(0xffffffffu, got);
+        if (!ok) break;
+        tc_fence_after();
+        // The row's BK scores of this block, loaded at once.
+        uint32_t r[BK];
+#pragma unroll
+        for (int q4 = 0; q4 < BK / 32; ++q4)
+          tmem_ld32(t_s + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
+        if constexpr (BK % 32 == 16) tmem_ld16(t_s + BK / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[BK / 32 * 32]));
+        tmem_ld_wait();
+        reg_fence(r);
+        if (j == j_last && valid_last < BK) {
+          // Key columns past the sequence end exist only in the last block.
+#pragma unroll
+          for (int i = 0; i < BK; ++i)
+            if (i >= valid_last) r[i] = f2u(-INFINITY);
+        }
+        float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
+#pragma unroll
+        for (int i = 4; i + 8 <= BK; i += 8) {
+          mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
+          mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
+          mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
+          mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
+        }
+        mx0 = fmax3(mx0, u2f(r[BK - 4]), u2f(r[BK - 3]));
+        mx1 = fmax3(mx1, u2f(r[BK - 2]), u2f(r[BK - 1]));
+        const float bmax = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+        s_best = fmaxf(s_best, bmax);
+        // The reference: the exact maximum on the first block; later it is
+        // raised only when the block's maximum exceeds it by more than the
+        // threshold (rare), and then O and l are rescaled (after the
+        // exponentials, with the scores no longer live; PV of the previous
+        // block is complete: its commit preceded this block's S, and this
+        // block's PV waits for the arrival below).
+        float alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m = bmax * c2;
+        } else {
+          const float m_cand = bmax * c2;
+          const bool raise = m_cand > m + kRescaleThreshold;
+          rescale = __any_sync(0xffffffffu, raise);
+          if (raise) {
+            alpha = ex2_approx(m - m_cand);
+            m = m_cand;
+          }
+        }
+        // p = 2^(s c2 - m) two columns at a time on the MUFU unit, stored as
+        // bf16 pairs over the first BK / 2 columns of S (already read).
+        const uint64_t negm = f2pack(-m, -m);
+        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+        auto chunk = [&](auto np_c, int e0, uint32_t (&pk)[decltype(np_c)::value]) {
+          constexpr int NP = decltype(np_c)::value;
+#pragma unroll
+          for (int i = 0; i < NP; ++i) {
+            const int e = e0 + 2 * i;
+            const uint64_t x = ffma2(f2pack(u2f(r[e]), u2f(r[e + 1])), c2x2, negm);
+            float xl, xh;
+            f2unpack(x, xl, xh);
+            const uint64_t pv = f2pack(ex2_approx(xl), ex2_approx(xh));
+            if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
+            float pl, ph;
+            f2unpack(pv, pl, ph);
+            pk[i] = pack_bf16x2(pl, ph);
+          }
+        };
+#pragma unroll
+        for (int c16 = 0; c16 < BK / 32; ++c16) {
+          uint32_t pk[16];
+          chunk(IntC<16>{}, c16 * 32, pk);
+          tmem_st16(t_s + c16 * 16, pk);
+        }
+        if constexpr (BK % 32 == 16) {
+          uint32_t pk[8];
+          chunk(IntC<8>{}, BK / 32 * 32, pk);
+          tmem_st8(t_s + BK / 32 * 16, pk);
+        }
+        if (rescale) {
+#pragma unroll
+          for (int q4 = 0; q4 < D / 32; ++q4) {
+            uint32_t ro[32];
+            tmem_ld32(t_o + q4 * 32, ro);
+            tmem_ld_wait();
+            reg_fence(ro);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ro[i] = f2u(u2f(ro[i]) * alpha);
+            tmem_st32(t_o + q4 * 32, ro);
+          }
+        }
+        float a0, a1, b0, b1;
+        f2unpack(acc0, a0, a1);
+        f2unpack(acc1, b0, b1);
+        l = l * alpha + ((a0 + a1) + (b0 + b1));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&c->p_full[slot]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l, LSE -------------------------------------------
+      // O holds sums of bf16-rounded probabilities while l sums the fp32 ones.
+      // Their mismatch is negligible except for a dominant probability, which
+      // is not exactly representable once the reference lags the row maximum
+      // (threshold above): the rounding error of the row's largest
+      // probability, re-formed here exactly as the softmax formed it, is moved
+      // into the normaliser, so that a row with one dominant key returns that
+      // key's value.  The largest score was exponentiated against the final
+      // reference m: a raise after its block needs a larger score.  The LSE
+      // keeps the fp32 sum.
+      const float p_best = ex2_approx(fmaf(s_best, c2, -m));
+      const float corr = __uint_as_float(pack_bf16x2(p_best, 0.f) << 16) - p_best;
+      const float l_o = l + corr;
+      const bool got = mbar_wait(&c->o_full[slot], tiles & 1, &c->abort, a.spin_ns);
+      ok = __all_sync(0xffffffffu, got) && ok;
+      if (!ok) break;
+      ++tiles;
+      tc_fence_after();
+      const bool pad_row = grow >= a.N;
+      const float inv_l = pad_row ? 0.f : 1.f / l_o;
+#pragma unroll
+      for (int q4 = 0; q4 < D / 32; ++q4) {
+        uint32_t ro[32];
+        tmem_ld32(t_o + q4 * 32, ro);
+        tmem_ld_wait();
+        reg_fence(ro);
+        uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 pk;
+          pk.x = pack_bf16x2(u2f(ro[8 * v4 + 0]) * inv_l, u2f(ro[8 * v4 + 1]) * inv_l);
+          pk.y = pack_bf16x2(u2f(ro[8 * v4 + 2]) * inv_l, u2f(ro[8 * v4 + 3]) * inv_l);
+          pk.z = pack_bf16x2(u2f(ro[8 * v4 + 4]) * inv_l, u2f(ro[8 * v4 + 5]) * inv_l);
+          pk.w = pack_bf16x2(u2f(ro[8 * v4 + 6]) * inv_l, u2f(ro[8 * v4 + 7]) * inv_l);
+          dst[v4] = pk;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&c->o_free[slot]);
+      if (a.lse != nullptr)
+        a.lse[orow_idx] = pad_row ? -INFINITY : (m + log2f(l)) * 0.69314718055994531f;
+    }
+    if (!ok) {
+      c->abort = 1;
+      report_status(a.status, CALIBATT_E_TIMEOUT);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kPpMma) tmem_dealloc(tmem, kTmemCols);
+}
+
 // SM count of every device, looked up on its first launch there.
 std::atomic<int> g_num_sms[kMaxDevices];
+
+// The two-slot kernel wherever its two slots fit in TMEM (all but d = 128 with
+// 144-key blocks); there the kernel that splits each block's keys between two
+// warps of the same rows.
+template <int D, int BK>
+constexpr bool kUsePp = (BK <= 128 ? 128 : 160) + D <= 256;
 
 template <int D, int BK>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
                cudaStream_t s) {
-  auto kern = k_attn_fwd<D, BK>;
-  constexpr uint32_t smem_bytes = FwdLayout<D, BK>::SMEM_BYTES;
+  constexpr bool pp = kUsePp<D, BK>;
+  auto kern = [] {
+    if constexpr (kUsePp<D, BK>) return k_attn_fwd_pp<D, BK>;
+    else return k_attn_fwd<D, BK>;
+  }();
+  constexpr uint32_t smem_bytes = [] {
+    if constexpr (kUsePp<D, BK>) return PpLayout<D, BK>::SMEM_BYTES;
+    else return FwdLayout<D, BK>::SMEM_BYTES;
+  }();
+  (void)pp;
   int dev = 0;
   if (int rc = current_device(&dev)) return rc;
   // One-time set-up per instantiation and device (the shared-memory limit is
