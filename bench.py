@@ -675,6 +675,12 @@ def other_workloads(device, pk):
     return rec
 
 
+def forward_kernel_name(d, bk):
+    """The forward kernel the library launches for head dim d and key-block size bk."""
+    two_slot = (128 if bk <= 128 else 160) + d <= 256
+    return f"k_attn_fwd_pp<{d}, {bk}>" if two_slot else f"k_attn_fwd<{d}, {bk}>"
+
+
 def kernel_traffic():
     """DRAM bytes per launch from the committed ncu capture, if the kernel source is unchanged."""
     if not TRAFFIC_FILE.exists():
@@ -804,7 +810,7 @@ def main_calibatt(args):
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_burst"],
                          "unit": UNIT, "frac": round(achieved / pk["bf16_burst"], 4),
                          "traffic": kernel_traffic(),
-                         "kernel": f"k_attn_fwd<{w.d}, {bk}>",
+                         "kernel": forward_kernel_name(w.d, bk),
                          "peak_kind": f"bf16_tflops, burst ({pk['source']}): each launch is a few ms and the timed "
                                       f"region well under the seconds-long loop of the sustained figure "
                                       f"({pk['bf16_sustained']})",
