@@ -692,18 +692,25 @@ struct PpLayout {
   static constexpr uint32_t QBOX_BYTES = TILE * 64 * 2;
   static constexpr uint32_t KBOX_BYTES = BK * 64 * 2;
   static constexpr uint32_t Q_BYTES = TILE * D * 2;
-  static constexpr uint32_t KV_BYTES = BK * D * 2;
-  static constexpr uint32_t OC = BK <= 128 ? 128 : 160;   // O_s column offset inside the slot
-  static_assert(BK % 16 == 0 && BK >= 64 && OC + D <= 256 && BK <= OC, "key-block size / head dim");
-  static_assert(KV_BYTES % 1024 == 0 && KBOX_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned tiles");
+  // 64-key blocks go two per step: one 128-key score tile whose halves hold
+  // two kept blocks (the second half repeats the first block, masked out,
+  // when a tile's count is odd), so the per-step costs are paid once per 128
+  // keys.
+  static constexpr int PAIR = BK == 64 ? 2 : 1;
+  static constexpr int SK = BK * PAIR;                    // keys per step
+  static constexpr uint32_t SBOX_BYTES = SK * 64 * 2;     // one 64-column box of a step's K or V tile
+  static constexpr uint32_t STEP_BYTES = SK * D * 2;      // a step's K (or V) tile
+  static constexpr uint32_t OC = SK <= 128 ? 128 : 160;   // O_s column offset inside the slot
+  static_assert(BK % 16 == 0 && BK >= 64 && OC + D <= 256 && SK <= OC, "key-block size / head dim");
+  static_assert(STEP_BYTES % 1024 == 0 && KBOX_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned tiles");
   static constexpr uint32_t OFF_Q = 0;   // Q tiles of slots 0 and 1
   static constexpr uint32_t OFF_RING = 2 * Q_BYTES;
   static constexpr uint32_t CTRL_BYTES = 1024;
   static constexpr uint32_t BUDGET = 232448 - OFF_RING - CTRL_BYTES - 1024;
-  // K/V tiles per slot ring (each slot's producer fills its own ring)
-  static constexpr int RING = (BUDGET / (2 * KV_BYTES)) > 4 ? 4 : static_cast<int>(BUDGET / (2 * KV_BYTES));
+  // K/V step tiles per slot ring (each slot's producer fills its own ring)
+  static constexpr int RING = (BUDGET / (2 * STEP_BYTES)) > 4 ? 4 : static_cast<int>(BUDGET / (2 * STEP_BYTES));
   static_assert(RING >= 2, "ring");
-  static constexpr uint32_t OFF_CTRL = OFF_RING + 2 * RING * KV_BYTES;
+  static constexpr uint32_t OFF_CTRL = OFF_RING + 2 * RING * STEP_BYTES;
   static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
 };
 
@@ -725,6 +732,21 @@ __device__ __forceinline__ void pp_cursor_init(const TcArgs& a, Cursor& cu, int 
 }
 
 constexpr int kPpProducer0 = 8, kPpMma = 9, kPpProducer1 = 11;   // warp 10 idle
+
+// Moves the cursor by `per` kept blocks (one step), to the next non-empty tile
+// of the walk when the current one is done.
+__device__ __forceinline__ void cursor_step(const TcArgs& a, Cursor& cu, int T, int stride, int per) {
+  cu.j += per;
+  if (cu.j >= cu.n) {
+    cu.t += stride;
+    cursor_seek(a, cu, T, stride);
+  }
+}
+
+// Key block at walk position j of the cursor's tile.
+__device__ __forceinline__ int cursor_kb_at(const TcArgs& a, const Cursor& cu, int j) {
+  return cu.base + a.pat_off[cu.p0 + (j + cu.rot) % cu.n];
+}
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -775,8 +797,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) regs_dec<kControlRegs>();
   if (warp == kPpProducer0 || warp == kPpProducer1) {
     // ===================== TMA producer of one slot ===========================
-    // Per kept block of the slot's walk: its K tile, then its V tile, into
-    // the slot's own ring (the order the slot's MMA warp consumes them).
+    // Per step of the slot's walk (one kept block, or two of 64 keys): its K
+    // tile, then its V tile, into the slot's own ring (the order the slot's MMA
+    // warp consumes them).
     const int s = warp == kPpProducer1;
     Cursor cu;
     pp_cursor_init(a, cu, s, T, G);
@@ -785,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const uint64_t pol = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
-    uint8_t* ring = smem + L::OFF_RING + s * R * L::KV_BYTES;
+    uint8_t* ring = smem + L::OFF_RING + s * R * L::STEP_BYTES;
     while (ok && !cu.done) {
       if (cu.j == 0) {
         ok = __all_sync(0xffffffffu, mbar_wait(&c->q_empty[s], (qf & 1) ^ 1, &c->abort, a.spin_ns));
@@ -798,19 +821,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++qf;
       }
       const int row = cu.bh * a.Npk + cursor_kb(a, cu) * BK;
+      // the step's second block (the first again when the count is odd)
+      const int row2 = (L::PAIR == 2 && cu.j + 1 < cu.n) ? cu.bh * a.Npk + cursor_kb_at(a, cu, cu.j + 1) * BK : row;
 #pragma unroll 1
       for (int kv = 0; kv < 2; ++kv) {
         const int e = g % R;
         ok = __all_sync(0xffffffffu, mbar_wait(&c->ring_empty[s][e], ((g / R) & 1) ^ 1, &c->abort, a.spin_ns));
         if (!ok) break;
-        mbar_arrive_expect_tx_w(&c->ring_full[s][e], L::KV_BYTES);
+        mbar_arrive_expect_tx_w(&c->ring_full[s][e], L::STEP_BYTES);
         const CUtensorMap* tm = kv ? &tmV : &tmK;
 #pragma unroll
-        for (int x = 0; x < D / 64; ++x)
-          tma_load_2d_w(ring + e * L::KV_BYTES + x * L::KBOX_BYTES, tm, x * 64, row, &c->ring_full[s][e], pol);
+        for (int x = 0; x < D / 64; ++x) {
+          tma_load_2d_w(ring + e * L::STEP_BYTES + x * L::SBOX_BYTES, tm, x * 64, row, &c->ring_full[s][e], pol);
+          if constexpr (L::PAIR == 2)
+            tma_load_2d_w(ring + e * L::STEP_BYTES + x * L::SBOX_BYTES + L::KBOX_BYTES, tm, x * 64, row2,
+                          &c->ring_full[s][e], pol);
+        }
         ++g;
       }
-      cursor_next(a, cu, T, 2 * G);
+      cursor_step(a, cu, T, 2 * G, L::PAIR);
     }
     if (lane == 0) {
       if (!ok) {
@@ -838,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor cu0, cu1;
     pp_cursor_init(a, cu0, 0, T, G);
     pp_cursor_init(a, cu1, 1, T, G);
-    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, BK, false);
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(TILE, L::SK, false);
     constexpr uint32_t IDESC_O = idesc_bf16_f32(TILE, D, true);
     uint32_t g0 = 0, g1 = 0;     // ring tiles consumed per slot
     uint32_t gb0 = 0, gb1 = 0;   // blocks whose PV was issued per slot
@@ -852,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Cursor& cu = s ? cu1 : cu0;
       uint32_t& g = s ? g1 : g0;
       int& qt = s ? qt1 : qt0;
-      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::KV_BYTES);
+      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::STEP_BYTES);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q + s * L::Q_BYTES);
       const uint32_t tS = tmem + s * 256;
       const int e = g % R;
@@ -860,21 +889,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                mbar_wait(&c->ring_full[s][e], (g / R) & 1, &c->abort, a.spin_ns);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      const uint32_t sK = sRing + e * L::KV_BYTES;
-      if (D == 128 && BK == TILE) {
+      const uint32_t sK = sRing + e * L::STEP_BYTES;
+      if (D == 128 && L::SK == TILE) {
         mma_ss_k128_w(tS, sdesc_sw128(sQ, 16, 1024), sdesc_sw128(sK, 16, 1024), IDESC_S, L::QBOX_BYTES >> 4);
       } else {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(sQ + (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + (kk >> 2) * L::SBOX_BYTES + (kk & 3) * 32, 16, 1024);
           mma_bf16_ss_w(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
         }
       }
       mma_commit_w(&c->s_full[s]);
       mma_commit_w(&c->ring_empty[s][e]);
       if (cu.j == 0) ++qt;
-      if (cu.j == cu.n - 1) mma_commit_w(&c->q_empty[s]);
+      if (cu.j + L::PAIR >= cu.n) mma_commit_w(&c->q_empty[s]);
       ++g;
       return true;
     };
@@ -885,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t& g = s ? g1 : g0;
       uint32_t& gb = s ? gb1 : gb0;
       int& ot = s ? ot1 : ot0;
-      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::KV_BYTES);
+      const uint32_t sRing = smem_u32(smem + L::OFF_RING + s * R * L::STEP_BYTES);
       const uint32_t tS = tmem + s * 256;
       const uint32_t tO = tS + OC;
       const int e = g % R;
@@ -893,22 +922,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                (cu.j > 0 || mbar_wait(&c->o_free[s], (ot & 1) ^ 1, &c->abort, a.spin_ns));
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      // P: BK / 2 columns of bf16 pairs at the start of S_s; 16 keys (8
+      // P: SK / 2 columns of bf16 pairs at the start of S_s; 16 keys (8
       // columns, 16 V rows = 2048 bytes) per K step.
-      const uint64_t vd = sdesc_sw128(sRing + e * L::KV_BYTES, L::KBOX_BYTES, 1024);
-      if (BK == TILE) {
+      const uint64_t vd = sdesc_sw128(sRing + e * L::STEP_BYTES, L::SBOX_BYTES, 1024);
+      if (L::SK == TILE) {
         mma_ts_k128_w(tO, tS, vd, IDESC_O, cu.j > 0 ? 1u : 0u);
       } else {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
+        for (int kk = 0; kk < L::SK / 16; ++kk)
           mma_bf16_ts_w(tO, tS + kk * 8, vd + kk * 128, IDESC_O, (cu.j > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit_w(&c->ring_empty[s][e]);
       if (cu.j == 0) ++ot;
-      if (cu.j == cu.n - 1) mma_commit_w(&c->o_full[s]);
+      if (cu.j + L::PAIR >= cu.n) mma_commit_w(&c->o_full[s]);
       ++g;
       ++gb;
-      cursor_next(a, cu, T, 2 * G);
+      cursor_step(a, cu, T, 2 * G, L::PAIR);
       return cu.done ? true : issue_s(s_c);
     };
     bool due0 = false, due1 = false;   // an S was issued whose PV is outstanding
@@ -968,35 +997,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY;
       float l = 0.f;
       float s_best = -INFINITY;   // largest raw score of the row (normalisation fix-up)
-      for (int j = 0; j < tl.n; ++j, ++gb) {
+      constexpr int SK = L::SK;
+      for (int j = 0; j < tl.n; j += L::PAIR, ++gb) {
         const bool got = mbar_wait(&c->s_full[slot], gb & 1, &c->abort, a.spin_ns);
         ok = __all_sync(0xffffffffu, got);
         if (!ok) break;
         tc_fence_after();
-        // The row's BK scores of this block, loaded at once.
-        uint32_t r[BK];
+        // The row's SK scores of this step, loaded at once.
+        uint32_t r[SK];
 #pragma unroll
-        for (int q4 = 0; q4 < BK / 32; ++q4)
+        for (int q4 = 0; q4 < SK / 32; ++q4)
           tmem_ld32(t_s + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
-        if constexpr (BK % 32 == 16) tmem_ld16(t_s + BK / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[BK / 32 * 32]));
+        if constexpr (SK % 32 == 16) tmem_ld16(t_s + SK / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[SK / 32 * 32]));
         tmem_ld_wait();
         reg_fence(r);
-        if (j == j_last && valid_last < BK) {
-          // Key columns past the sequence end exist only in the last block.
+        // Key columns past the sequence end exist only in the highest kept
+        // block; with two blocks per step, a step of one block masks its
+        // second half (the first block repeated) entirely.
+        int lim0 = BK, lim1 = BK;
+        if (j == j_last) lim0 = valid_last;
+        if constexpr (L::PAIR == 2) {
+          if (j + 1 >= tl.n) lim1 = 0;
+          else if (j + 1 == j_last) lim1 = valid_last;
+        }
+        if (lim0 < BK || lim1 < BK) {
 #pragma unroll
-          for (int i = 0; i < BK; ++i)
-            if (i >= valid_last) r[i] = f2u(-INFINITY);
+          for (int i = 0; i < SK; ++i)
+            if (i < BK ? i >= lim0 : i - BK >= lim1) r[i] = f2u(-INFINITY);
         }
         float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
 #pragma unroll
-        for (int i = 4; i + 8 <= BK; i += 8) {
+        for (int i = 4; i + 8 <= SK; i += 8) {
           mx0 = fmax3(mx0, u2f(r[i + 0]), u2f(r[i + 1]));
           mx1 = fmax3(mx1, u2f(r[i + 2]), u2f(r[i + 3]));
           mx2 = fmax3(mx2, u2f(r[i + 4]), u2f(r[i + 5]));
           mx3 = fmax3(mx3, u2f(r[i + 6]), u2f(r[i + 7]));
         }
-        mx0 = fmax3(mx0, u2f(r[BK - 4]), u2f(r[BK - 3]));
-        mx1 = fmax3(mx1, u2f(r[BK - 2]), u2f(r[BK - 1]));
+        mx0 = fmax3(mx0, u2f(r[SK - 4]), u2f(r[SK - 3]));
+        mx1 = fmax3(mx1, u2f(r[SK - 2]), u2f(r[SK - 1]));
         const float bmax = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         s_best = fmaxf(s_best, bmax);
         // The reference: the exact maximum on the first block; later it is
@@ -1019,7 +1057,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         // p = 2^(s c2 - m) two columns at a time on the MUFU unit, stored as
-        // bf16 pairs over the first BK / 2 columns of S (already read).
+        // bf16 pairs over the first SK / 2 columns of S (already read).
         const uint64_t negm = f2pack(-m, -m);
         uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
         auto chunk = [&](auto np_c, int e0, uint32_t (&pk)[decltype(np_c)::value]) {
@@ -1038,15 +1076,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
 #pragma unroll
-        for (int c16 = 0; c16 < BK / 32; ++c16) {
+        for (int c16 = 0; c16 < SK / 32; ++c16) {
           uint32_t pk[16];
           chunk(IntC<16>{}, c16 * 32, pk);
           tmem_st16(t_s + c16 * 16, pk);
         }
-        if constexpr (BK % 32 == 16) {
+        if constexpr (SK % 32 == 16) {
           uint32_t pk[8];
-          chunk(IntC<8>{}, BK / 32 * 32, pk);
-          tmem_st8(t_s + BK / 32 * 16, pk);
+          chunk(IntC<8>{}, SK / 32 * 32, pk);
+          tmem_st8(t_s + SK / 32 * 16, pk);
         }
         if (rescale) {
 #pragma unroll
