@@ -292,6 +292,35 @@ def test_bf16_key_blocks_of_64(d):
     run_k64_compare(q, k, v, mask, N, d)
 
 
+@pytest.mark.parametrize("N", [2000, 1985])
+def test_bf16_key_blocks_of_64_pairs(N):
+    # 64-key blocks are computed two per step: rows with 1, 2 and 3 kept
+    # blocks (a last step holding one block), the partial last key block
+    # (N = 2000: 16 real keys in block 31; N = 1985: 1 real key) walked in the
+    # first half of a step, in the second half and alone, and rows whose walk
+    # wraps around from their diagonal block.
+    d, Np, H = 128, 2048, 2
+    q, k, v = syn.normal_qkv(1, H, N, Np, d, 63)
+    mask = np.zeros((H, 16, 32), np.uint8)
+    # head 0: the row's own (diagonal) block is walked first
+    mask[0, 0, [0]] = 1                       # one block
+    mask[0, 1, [2, 3]] = 1                    # one full step
+    mask[0, 2, [4, 9, 20]] = 1                # a step and a single block
+    mask[0, 3, [31]] = 1                      # the partial block alone
+    mask[0, 4, [8, 31]] = 1                   # partial block in the second half
+    mask[0, 5, [31, 3]] = 1                   # diagonal 10: walk 31, then 3 (partial block first half)
+    mask[0, 6, [12, 13, 31]] = 1              # partial block in a single-block last step
+    mask[0, 15, [30, 31]] = 1                 # diagonal 30: 30, 31
+    mask[0, 14, [0, 5, 28, 29, 31]] = 1       # odd count with wrap-around
+    # head 1: random odd and even counts, last block always kept
+    rng = np.random.default_rng(64)
+    mask[1] = (rng.random((16, 32)) < 0.2).astype(np.uint8)
+    mask[1, :, 31] = 1
+    mask[1, 3, :] = 0
+    mask[1, 3, 7] = 1
+    run_k64_compare(q, k, v, mask, N, d)
+
+
 def test_bf16_key_blocks_of_64_large_score_jumps():
     # The redo / O-rescale paths with 64-key blocks (magnitudes set per
     # 32-key quarter block, so jumps fall in both halves of a block).
