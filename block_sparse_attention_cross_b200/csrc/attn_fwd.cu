@@ -918,10 +918,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tS = tmem + s * 256;
       const uint32_t tO = tS + OC;
       const int e = g % R;
-      bool w = mbar_wait(&c->ring_full[s][e], (g / R) & 1, &c->abort, a.spin_ns) &&
-               (cu.j > 0 || mbar_wait(&c->o_free[s], (ot & 1) ^ 1, &c->abort, a.spin_ns));
-      if (!__all_sync(0xffffffffu, w)) return false;
-      tc_fence_after();
       // P: SK / 2 columns of bf16 pairs at the start of S_s; 16 keys (8
       // columns, 16 V rows = 2048 bytes) per K step.
       const uint64_t vd = sdesc_sw128(sRing + e * L::STEP_BYTES, L::SBOX_BYTES, 1024);
@@ -947,8 +943,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && (due0 || due1)) {
       // the slots in turn (suspending waits)
       const int s = (due0 && (turn == 0 || !due1)) ? 0 : 1;
-      const bool w = mbar_wait(&c->p_full[s], (s ? gb1 : gb0) & 1, &c->abort, a.spin_ns);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      // The PV's V tile and (first block of a tile) the free O are usually
+      // ready long before P: wait for them first, so that only P stands
+      // between the softmax's last store and the PV issue.
+      {
+        const Cursor& cu = s ? cu1 : cu0;
+        const uint32_t g = s ? g1 : g0;
+        const int ot = s ? ot1 : ot0;
+        const bool w = mbar_wait(&c->ring_full[s][g % R], (g / R) & 1, &c->abort, a.spin_ns) &&
+                       (cu.j > 0 || mbar_wait(&c->o_free[s], (ot & 1) ^ 1, &c->abort, a.spin_ns)) &&
+                       mbar_wait(&c->p_full[s], (s ? gb1 : gb0) & 1, &c->abort, a.spin_ns);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      }
       tc_fence_after();
       if (s == 0) {
         ok = issue_pv(IntC<0>{});
