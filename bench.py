@@ -47,7 +47,7 @@ import statistics
 import subprocess
 import sys
 import time
-from datetime import timedelta
+from datetime import datetime, timedelta
 from pathlib import Path
 
 import numpy as np
@@ -206,23 +206,40 @@ def cpu_model():
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 25 ms, timestamped) kept for the timed window only.
+
+    start() waits for the first sample, so the sampler is running before the
+    caller's warm-up; mark_window(t0, t1) records the timed region's host wall
+    times, and stop() keeps the samples inside it (or, if the region was
+    shorter than the sampling period, the samples nearest to it)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.window = None
         self.path = Path(os.environ.get("TMPDIR", "/tmp")) / f"calibatt_clocks_{os.getpid()}.csv"
 
     def start(self):
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "25"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+            return
+        deadline = time.time() + 5.0
+        while time.time() < deadline and self.proc.poll() is None:
+            self.fh.flush()
+            if self.path.stat().st_size > 0:
+                break
+            time.sleep(0.01)
+
+    def mark_window(self, t0, t1):
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
@@ -236,16 +253,24 @@ class ClockSampler:
         rows = []
         for line in self.path.read_text().splitlines():
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
-                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7], "power_cap": parts[8]})
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append({"t": ts, "sm": float(parts[2]), "max": float(parts[3]), "power": float(parts[4]),
+                             "hw": parts[6], "hw_thermal": parts[7], "sw_thermal": parts[8], "power_cap": parts[9]})
             except ValueError:
                 continue
         self.path.unlink(missing_ok=True)
         if not rows:
             return None
+        in_window = rows
+        if self.window is not None:
+            t0, t1 = self.window
+            in_window = [r for r in rows if t0 <= r["t"] <= t1]
+            if not in_window:   # region shorter than the period: the samples nearest to it
+                in_window = sorted(rows, key=lambda r: min(abs(r["t"] - t0), abs(r["t"] - t1)))[:2]
+        rows = in_window
         load = [r for r in rows if r["power"] > 200.0] or rows
         reasons = set()
         for r in load:
@@ -722,11 +747,14 @@ def main_calibatt(args):
     warm = max(3, args.warmup)
     launches0 = cba.launch_count()
     clocks = ClockSampler(physical_gpu_id(local))
+    clocks.start()
     for _ in range(warm):
         step()
     launches_warm = cba.launch_count()
-    clocks.start()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
     total_ms, per = time_calls(step, args.steps, 0, torch, dist)
+    clocks.mark_window(t_wall0, time.time())
     clk = clocks.stop()
     launches = cba.launch_count() - launches_warm
     t_max = max_over_ranks(total_ms, dist, dev)
