@@ -58,7 +58,7 @@ UNIT = "TFLOP/s"
 WORKLOAD = "wan480_25"
 KERNEL_SOURCE = ROOT / "block_sparse_attention_cross_b200" / "csrc" / "attn_fwd.cu"
 TRAFFIC_FILE = ROOT / "profiles" / "traffic.json"
-E2E_HEADS_PER_CHUNK = 4
+E2E_HEADS_PER_CHUNK = 2
 
 
 def parse_args(argv=None):

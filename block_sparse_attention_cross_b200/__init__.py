@@ -199,7 +199,7 @@ def _need_host(*ts):
             raise ValueError("host tensors must be contiguous CPU tensors (pin_memory() for overlap)")
 
 
-def sparse_attn_fwd_streamed(q, k, v, bl: BlockList, N, staging, scale=None, map_offset=0, heads_per_chunk=8,
+def sparse_attn_fwd_streamed(q, k, v, bl: BlockList, N, staging, scale=None, map_offset=0, heads_per_chunk=2,
                              out=None, lse=None, status=None):
     """Block-sparse attention forward for q, k, v in host memory.
 
