@@ -11,13 +11,19 @@
 // to three key blocks, whose boundaries fall on 16-column chunks, so every
 // chunk's sum goes to exactly one block.
 //
-// CTA = one 128-row query tile of one head, 8 warps:
+// CTA = one 128-row query tile of one head, 12 warps:
 //   warp 0      TMA producer: the Q tile once, then every K tile into a
 //               4-deep ring.
 //   warp 1      TMEM allocator and MMA issuer: S = Q K^T into one of two TMEM
 //               S buffers (columns [0,128) and [128,256)), so the next block's
 //               product overlaps the current block's exponentials.
-//   warps 4..7  score warpgroup: thread t owns query row t (TMEM lane t).
+//   warps 4..7  score warpgroup 0: key columns [0, 64) of every tile; thread t
+//               owns query row t (TMEM lane t).
+//   warps 8..11 score warpgroup 1: key columns [64, 128) of the same rows.
+// Both passes are MUFU-bound (one exponential per score); two score warps per
+// SM sub-partition keep that unit busy.  The energy pass needs no exchange
+// between the halves (row sums per key block are reduced over rows anyway);
+// the statistics pass merges the halves' (max, sum) once per tile.
 // Both control warps run their loops warp-uniformly and issue through one
 // elected lane.  Every wait is bounded; on expiry the CTA records
 // CALIBATT_E_TIMEOUT, waits (bounded) for its own copies and MMAs, frees TMEM
@@ -34,7 +40,7 @@ namespace {
 enum { MODE_STATS = 1, MODE_ENERGY = 2 };
 
 constexpr int TILE = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kRing = 4;
 constexpr int kMaxBlocks = 2048;  // key blocks per row (partials buffer)
@@ -45,8 +51,9 @@ struct EnergyLayout {
   static constexpr uint32_t TILE_BYTES = TILE * D * 2;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + TILE_BYTES;
-  static constexpr uint32_t OFF_PART = OFF_K + kRing * TILE_BYTES;   // ENERGY: per-warp block sums
-  static constexpr uint32_t OFF_CTRL = OFF_PART + kMaxBlocks * 4 * 4;
+  // ENERGY: per-warp block sums, 8 per key block; STATS: the halves' (max, sum) per row
+  static constexpr uint32_t OFF_PART = OFF_K + kRing * TILE_BYTES;
+  static constexpr uint32_t OFF_CTRL = OFF_PART + kMaxBlocks * 8 * 4;
   static constexpr uint32_t CTRL_BYTES = 1024;
   static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
 };
@@ -88,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&c->s_full[s], 1);
-      mbar_init(&c->s_empty[s], 128);
+      mbar_init(&c->s_empty[s], 256);
     }
     mbar_init(&c->drain, 1);
     c->abort = 0;
@@ -165,8 +172,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_commit_w(&c->drain);
     mbar_wait(&c->drain, 0, nullptr, a.spin_ns);
   } else if (warp >= 4) {
-    // ===================== score warpgroup ===================================
-    const int w = warp - 4;
+    // ===================== score warpgroups ==================================
+    const int w = warp & 3;                   // TMEM lane quarter
+    const int hh = (warp - 4) >> 2;           // key-column half of every tile
+    const int c0 = hh * 64;
+    const int w8 = hh * 4 + w;                // this warp's partial slot
     const int row = w * 32 + lane;
     const int grow = qb * TILE + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(w * 32) << 16);
@@ -174,8 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* part = reinterpret_cast<float*>(smem + L::OFF_PART);
     const int bk = a.block_k;
     if (MODE == MODE_ENERGY && bk != TILE) {
-      // Each warp owns the slots part[4 * kb + w]; they accumulate across tiles.
-      for (int kb = lane; kb < a.nke; kb += 32) part[4 * kb + w] = 0.f;
+      // Each warp owns the slots part[8 * kb + w8]; they accumulate across tiles.
+      for (int kb = lane; kb < a.nke; kb += 32) part[8 * kb + w8] = 0.f;
       __syncwarp();
     }
     const float lse2_row =
@@ -188,16 +198,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&c->s_full[sb], (j >> 1) & 1, &c->abort, a.spin_ns));
       if (!ok) break;
       tc_fence_after();
-      float s[TILE];
+      float s[64];
       {
-        uint32_t r[TILE];
+        uint32_t r[64];
 #pragma unroll
-        for (int q4 = 0; q4 < TILE / 32; ++q4)
-          tmem_ld32(t_lane + sb * TILE + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
+        for (int q4 = 0; q4 < 2; ++q4)
+          tmem_ld32(t_lane + sb * TILE + c0 + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[q4 * 32]));
         tmem_ld_wait();
         reg_fence(r);
 #pragma unroll
-        for (int i = 0; i < TILE; ++i) s[i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(r[i]);
       }
       tc_fence_before();
       mbar_arrive(&c->s_empty[sb]);
@@ -205,18 +215,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int valid = (j == a.nkb - 1) ? (a.N - j * TILE) : TILE;
       if (valid < TILE) {
 #pragma unroll
-        for (int i = 0; i < TILE; ++i)
-          if (i >= valid) s[i] = -INFINITY;
+        for (int i = 0; i < 64; ++i)
+          if (c0 + i >= valid) s[i] = -INFINITY;
       }
       if (MODE == MODE_ENERGY && bk == TILE) {
         float rs = 0.f;
         if (grow < a.N) {
 #pragma unroll
-          for (int i = 0; i < TILE; ++i) rs += ex2_approx(fmaf(s[i], c2, -lse2_row));
+          for (int i = 0; i < 64; ++i) rs += ex2_approx(fmaf(s[i], c2, -lse2_row));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-        if (lane == 0) part[j * 4 + w] = rs;
+        if (lane == 0) part[j * 8 + w8] = rs;
       } else if (MODE == MODE_ENERGY) {
         // Key blocks kb0, kb0+1, kb0+2 meet this tile at columns [0,b1),
         // [b1,b2), [b2,128); b1 and b2 are multiples of 16.
@@ -226,12 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float r0 = 0.f, r1 = 0.f, r2 = 0.f;
         if (grow < a.N) {
 #pragma unroll
-          for (int c = 0; c < TILE / 16; ++c) {
+          for (int cc = 0; cc < 4; ++cc) {
             float cs = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) cs += ex2_approx(fmaf(s[c * 16 + i], c2, -lse2_row));
-            if (c * 16 < b1) r0 += cs;
-            else if (c * 16 < b2) r1 += cs;
+            for (int i = 0; i < 16; ++i) cs += ex2_approx(fmaf(s[cc * 16 + i], c2, -lse2_row));
+            const int col = c0 + cc * 16;
+            if (col < b1) r0 += cs;
+            else if (col < b2) r1 += cs;
             else r2 += cs;
           }
         }
@@ -242,39 +253,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           r2 += __shfl_xor_sync(0xffffffffu, r2, o);
         }
         if (lane == 0) {
-          part[4 * kb0 + w] += r0;
-          if (b1 < TILE && kb0 + 1 < a.nke) part[4 * (kb0 + 1) + w] += r1;
-          if (b2 < TILE && kb0 + 2 < a.nke) part[4 * (kb0 + 2) + w] += r2;
+          part[8 * kb0 + w8] += r0;
+          if (b1 < TILE && kb0 + 1 < a.nke) part[8 * (kb0 + 1) + w8] += r1;
+          if (b2 < TILE && kb0 + 2 < a.nke) part[8 * (kb0 + 2) + w8] += r2;
         }
         __syncwarp();
       } else {
         float mx = s[0];
 #pragma unroll
-        for (int i = 1; i < TILE; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 1; i < 64; ++i) mx = fmaxf(mx, s[i]);
         const float m_new = fmaxf(m, mx * c2);
-        const float alpha = ex2_approx(m - m_new);
-        const float neg = -m_new;
-        float rs = 0.f;
+        // (a half whose columns are all past the sequence end so far keeps m = -inf)
+        if (m_new != -INFINITY) {
+          const float alpha = ex2_approx(m - m_new);
+          const float neg = -m_new;
+          float rs = 0.f;
 #pragma unroll
-        for (int i = 0; i < TILE; ++i) rs += ex2_approx(fmaf(s[i], c2, neg));
-        l = l * alpha + rs;
-        m = m_new;
+          for (int i = 0; i < 64; ++i) rs += ex2_approx(fmaf(s[i], c2, neg));
+          l = l * alpha + rs;
+          m = m_new;
+        }
       }
     }
     if (!ok) give_up(c, a.status);
     if (MODE == MODE_STATS) {
-      a.lse2[static_cast<size_t>(h) * a.Np + grow] = (ok && grow < a.N) ? m + log2f(l) : -INFINITY;
+      // The two halves of each row: (max, sum) merged in half 0.
+      float2* xb = reinterpret_cast<float2*>(smem + L::OFF_PART);
+      xb[hh * 128 + row] = make_float2(m, l);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (hh == 0) {
+        const float2 o = xb[128 + row];
+        const float mm = fmaxf(m, o.x);
+        float ll = 0.f;
+        if (mm != -INFINITY) ll = l * ex2_approx(m - mm) + o.y * ex2_approx(o.x - mm);
+        a.lse2[static_cast<size_t>(h) * a.Np + grow] = (ok && grow < a.N && mm != -INFINITY) ? mm + log2f(ll) : -INFINITY;
+      }
     } else {
-      // ENERGY: per key block, the four warp partials in a fixed order.
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // ENERGY: per key block, the eight warp partials in a fixed order.
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       if (ok) {
         const int rows = min(TILE, a.N - qb * TILE);
         const float inv_rows = 1.f / static_cast<float>(rows);
         const int ne = (bk == TILE) ? n : a.nke;
         float* erow = a.energy + (static_cast<size_t>(h) * a.nqb + qb) * ne;
-        for (int j = row; j < ne; j += TILE) {
-          const float tot = ((part[4 * j + 0] + part[4 * j + 1]) + part[4 * j + 2]) + part[4 * j + 3];
-          erow[j] = tot * inv_rows;
+        for (int jj = hh * 128 + row; jj < ne; jj += 256) {
+          const float* pp = part + 8 * jj;
+          const float tot = ((pp[0] + pp[1]) + (pp[2] + pp[3])) + ((pp[4] + pp[5]) + (pp[6] + pp[7]));
+          erow[jj] = tot * inv_rows;
         }
       }
     }
