@@ -218,12 +218,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 64; ++i)
           if (c0 + i >= valid) s[i] = -INFINITY;
       }
+      // sum of 2^(s c2 - ref) over columns [i0, i0 + 2 np): packed pairs, two
+      // accumulators (independent chains for the MUFU pipe)
+      const uint64_t c2x2 = f2pack(c2, c2);
+      auto exp_sum = [&](int i0, int np, float ref) {
+        const uint64_t negr = f2pack(-ref, -ref);
+        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+        for (int i = 0; i < np; ++i) {
+          const uint64_t x = ffma2(f2pack(s[i0 + 2 * i], s[i0 + 2 * i + 1]), c2x2, negr);
+          float xl, xh;
+          f2unpack(x, xl, xh);
+          const uint64_t pv = f2pack(ex2_approx(xl), ex2_approx(xh));
+          if (i & 1) acc1 = fadd2(acc1, pv); else acc0 = fadd2(acc0, pv);
+        }
+        float a0, a1, b0, b1;
+        f2unpack(acc0, a0, a1);
+        f2unpack(acc1, b0, b1);
+        return (a0 + a1) + (b0 + b1);
+      };
       if (MODE == MODE_ENERGY && bk == TILE) {
         float rs = 0.f;
-        if (grow < a.N) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) rs += ex2_approx(fmaf(s[i], c2, -lse2_row));
-        }
+        if (grow < a.N) rs = exp_sum(0, 32, lse2_row);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
         if (lane == 0) part[j * 8 + w8] = rs;
@@ -237,9 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (grow < a.N) {
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
-            float cs = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) cs += ex2_approx(fmaf(s[cc * 16 + i], c2, -lse2_row));
+            const float cs = exp_sum(cc * 16, 8, lse2_row);
             const int col = c0 + cc * 16;
             if (col < b1) r0 += cs;
             else if (col < b2) r1 += cs;
@@ -259,18 +273,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       } else {
-        float mx = s[0];
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int i = 1; i < 64; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 4; i < 60; i += 8) {
+          mx0 = fmax3(mx0, s[i], s[i + 1]);
+          mx1 = fmax3(mx1, s[i + 2], s[i + 3]);
+          mx2 = fmax3(mx2, s[i + 4], s[i + 5]);
+          mx3 = fmax3(mx3, s[i + 6], s[i + 7]);
+        }
+        mx0 = fmax3(mx0, s[60], s[61]);
+        mx1 = fmax3(mx1, s[62], s[63]);
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float m_new = fmaxf(m, mx * c2);
         // (a half whose columns are all past the sequence end so far keeps m = -inf)
         if (m_new != -INFINITY) {
           const float alpha = ex2_approx(m - m_new);
-          const float neg = -m_new;
-          float rs = 0.f;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) rs += ex2_approx(fmaf(s[i], c2, neg));
-          l = l * alpha + rs;
+          l = l * alpha + exp_sum(0, 32, m_new);
           m = m_new;
         }
       }
