@@ -40,7 +40,7 @@ namespace calibatt {
 namespace {
 
 constexpr int TILE = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRing = 4;
 
@@ -51,7 +51,8 @@ struct SimLayout {
   static constexpr uint32_t OFF_Q = 0;                          // Q, then Q'
   static constexpr uint32_t OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr uint32_t OFF_RED = OFF_K + kRing * TILE_BYTES;   // 4 warp partial sums + counts
-  static constexpr uint32_t OFF_CTRL = OFF_RED + 64;
+  static constexpr uint32_t OFF_HALF = OFF_RED + 64;   // column half 1's (dot, |a|^2, |b|^2) per row
+  static constexpr uint32_t OFF_CTRL = OFF_HALF + TILE * 3 * 4;
   static constexpr uint32_t CTRL_BYTES = 512;
   static constexpr uint32_t SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;
 };
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&c->s_full[s], 1);
-      mbar_init(&c->s_empty[s], 128);
+      mbar_init(&c->s_empty[s], 256);
     }
     mbar_init(&c->drain, 1);
     c->abort = 0;
@@ -189,8 +190,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_commit_w(&c->drain);
     mbar_wait(&c->drain, 0, nullptr, a.spin_ns);
   } else if (warp >= 4) {
-    // ===================== row warpgroup =====================================
-    const int w = warp - 4;
+    // ===================== row warpgroups ====================================
+    // Warps 4-7 take key columns [0, 64) of every block, warps 8-11 [64, 128)
+    // (two warps per SM sub-partition for the MUFU unit); half 1 hands its
+    // row sums to half 0, which forms the cosine.
+    const int w = warp & 3;
+    const int hh = (warp - 4) >> 2;
+    const int c0 = hh * 64;
     const int row = w * 32 + lane;
     const int grow = qb * TILE + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(w * 32) << 16);
@@ -206,31 +212,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int valid = (j == a.nkb - 1) ? (a.N - j * TILE) : TILE;   // real keys of this block
-      float dot_b = 0.f, na_b = 0.f, nb_b = 0.f;   // this block's sums, added to the row's totals after it
+      // this block's sums (two accumulators each), added to the row's totals after it
+      float dot0 = 0.f, na0 = 0.f, nb0 = 0.f, dot1 = 0.f, na1 = 0.f, nb1 = 0.f;
 #pragma unroll
-      for (int q4 = 0; q4 < TILE / 32; ++q4) {
+      for (int q4 = 0; q4 < 2; ++q4) {
         uint32_t ra[32], rb[32];
-        tmem_ld32(t_lane + sb * 256 + q4 * 32, ra);
-        tmem_ld32(t_lane + sb * 256 + TILE + q4 * 32, rb);
+        tmem_ld32(t_lane + sb * 256 + c0 + q4 * 32, ra);
+        tmem_ld32(t_lane + sb * 256 + TILE + c0 + q4 * 32, rb);
         tmem_ld_wait();
         reg_fence(ra);
         reg_fence(rb);
         if (counted) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (q4 * 32 + i < valid) {
+            if (c0 + q4 * 32 + i < valid) {
               const float pa = ex2_approx(fmaf(__uint_as_float(ra[i]), c2, -lse_a));
               const float pb = ex2_approx(fmaf(__uint_as_float(rb[i]), c2, -lse_b));
-              dot_b = fmaf(pa, pb, dot_b);
-              na_b = fmaf(pa, pa, na_b);
-              nb_b = fmaf(pb, pb, nb_b);
+              if (i & 1) {
+                dot1 = fmaf(pa, pb, dot1);
+                na1 = fmaf(pa, pa, na1);
+                nb1 = fmaf(pb, pb, nb1);
+              } else {
+                dot0 = fmaf(pa, pb, dot0);
+                na0 = fmaf(pa, pa, na0);
+                nb0 = fmaf(pb, pb, nb0);
+              }
             }
           }
         }
       }
-      dot += dot_b;
-      na += na_b;
-      nb += nb_b;
+      dot += dot0 + dot1;
+      na += na0 + na1;
+      nb += nb0 + nb1;
       tc_fence_before();
       mbar_arrive(&c->s_empty[sb]);
     }
@@ -238,24 +251,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       c->abort = 1;
       report_status(a.status, CALIBATT_E_TIMEOUT);
     }
-    // Fixed-order reduction of the tile: lanes by shuffle, then the 4 warps.
-    float cs = (counted && na > 0.f && nb > 0.f) ? dot * rsqrtf(na * nb) : 0.f;
-    int cnt = counted ? 1 : 0;
+    // The row's sums: half 0's plus half 1's, in that order.
+    float* half = reinterpret_cast<float*>(smem + L::OFF_HALF);
+    if (hh == 1) {
+      half[row] = dot;
+      half[TILE + row] = na;
+      half[2 * TILE + row] = nb;
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (hh == 0) {
+      dot += half[row];
+      na += half[TILE + row];
+      nb += half[2 * TILE + row];
+      // Fixed-order reduction of the tile: lanes by shuffle, then the 4 warps.
+      float cs = (counted && na > 0.f && nb > 0.f) ? dot * rsqrtf(na * nb) : 0.f;
+      int cnt = counted ? 1 : 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      cs += __shfl_xor_sync(0xffffffffu, cs, o);
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    }
-    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
-    int* redc = reinterpret_cast<int*>(smem + L::OFF_RED + 32);
-    if (lane == 0) {
-      red[w] = cs;
-      redc[w] = cnt;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (row == 0 && ok) {
-      a.tile_sum[h * a.nqb + qb] = ((red[0] + red[1]) + red[2]) + red[3];
-      a.tile_cnt[h * a.nqb + qb] = redc[0] + redc[1] + redc[2] + redc[3];
+      for (int o = 16; o > 0; o >>= 1) {
+        cs += __shfl_xor_sync(0xffffffffu, cs, o);
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      }
+      float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
+      int* redc = reinterpret_cast<int*>(smem + L::OFF_RED + 32);
+      if (lane == 0) {
+        red[w] = cs;
+        redc[w] = cnt;
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (row == 0 && ok) {
+        a.tile_sum[h * a.nqb + qb] = ((red[0] + red[1]) + red[2]) + red[3];
+        a.tile_cnt[h * a.nqb + qb] = redc[0] + redc[1] + redc[2] + redc[3];
+      }
     }
   }
 
