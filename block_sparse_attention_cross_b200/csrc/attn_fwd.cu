@@ -687,22 +687,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 // scores of block j + 1 are visible.
 // ===========================================================================
 
+constexpr int cgcd(int x, int y) { return y == 0 ? x : cgcd(y, x % y); }
+
 template <int D, int BK>
 struct PpLayout {
   static constexpr uint32_t QBOX_BYTES = TILE * 64 * 2;
   static constexpr uint32_t KBOX_BYTES = BK * 64 * 2;
   static constexpr uint32_t Q_BYTES = TILE * D * 2;
-  // 64-key blocks go two per step: one 128-key score tile whose halves hold
-  // two kept blocks (the second half repeats the first block, masked out,
-  // when a tile's count is odd), so the per-step costs are paid once per 128
-  // keys.
-  static constexpr int PAIR = BK == 64 ? 2 : 1;
-  static constexpr int SK = BK * PAIR;                    // keys per step
+  // Steps of 128 keys where gcd(BK, 128) >= 32 (BK = 64, 96, 128): the keys
+  // come in pieces of PK = gcd(BK, 128), taken in walk order from the kept
+  // blocks (a block is BK / PK pieces, a step 128 / PK: one block at 128, two
+  // at 64, parts of two at 96), one TMA box per piece and 64 columns; the last
+  // step of a tile repeats its last real piece where the walk has ended, and
+  // the softmax masks those columns.  So each step pays its fixed costs once
+  // per 128 keys.  With 16-key pieces (BK = 80, 144) the many small copies
+  // cost more than they save (measured: -8% and -12%), so there a step is one
+  // block.
+  static constexpr int PG = cgcd(BK, TILE);
+  static constexpr bool PACK = PG >= 32;
+  static constexpr int PK = PACK ? PG : BK;               // keys per piece
+  static constexpr int SK = PACK ? TILE : BK;             // keys per step
+  static constexpr int PPB = BK / PK;                     // pieces per key block
+  static constexpr int PPS = SK / PK;                     // pieces per step
+  static constexpr uint32_t PBOX_BYTES = PK * 64 * 2;     // one 64-column box of a piece (one TMA copy)
   static constexpr uint32_t SBOX_BYTES = SK * 64 * 2;     // one 64-column box of a step's K or V tile
   static constexpr uint32_t STEP_BYTES = SK * D * 2;      // a step's K (or V) tile
   static constexpr uint32_t OC = SK <= 128 ? 128 : 160;   // O_s column offset inside the slot
   static_assert(BK % 16 == 0 && BK >= 64 && OC + D <= 256 && SK <= OC, "key-block size / head dim");
-  static_assert(STEP_BYTES % 1024 == 0 && KBOX_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned tiles");
+  static_assert(PBOX_BYTES % 1024 == 0 && STEP_BYTES % 1024 == 0, "128-byte swizzle needs 1 KB aligned boxes");
   static constexpr uint32_t OFF_Q = 0;   // Q tiles of slots 0 and 1
   static constexpr uint32_t OFF_RING = 2 * Q_BYTES;
   static constexpr uint32_t CTRL_BYTES = 1024;
@@ -733,11 +745,12 @@ __device__ __forceinline__ void pp_cursor_init(const TcArgs& a, Cursor& cu, int 
 
 constexpr int kPpProducer0 = 8, kPpMma = 9, kPpProducer1 = 11;   // warp 10 idle
 
-// Moves the cursor by `per` kept blocks (one step), to the next non-empty tile
-// of the walk when the current one is done.
-__device__ __forceinline__ void cursor_step(const TcArgs& a, Cursor& cu, int T, int stride, int per) {
+// Moves a piece cursor (cu.j counts pieces, ppb per kept block) by `per`
+// pieces (one step), to the next non-empty tile of the walk when the current
+// one is done.
+__device__ __forceinline__ void cursor_step(const TcArgs& a, Cursor& cu, int T, int stride, int per, int ppb) {
   cu.j += per;
-  if (cu.j >= cu.n) {
+  if (cu.j >= cu.n * ppb) {
     cu.t += stride;
     cursor_seek(a, cu, T, stride);
   }
@@ -797,9 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) regs_dec<kControlRegs>();
   if (warp == kPpProducer0 || warp == kPpProducer1) {
     // ===================== TMA producer of one slot ===========================
-    // Per step of the slot's walk (one kept block, or two of 64 keys): its K
-    // tile, then its V tile, into the slot's own ring (the order the slot's MMA
-    // warp consumes them).
+    // Per step of the slot's walk (128 keys in pieces from the kept blocks):
+    // its K tile, then its V tile, into the slot's own ring (the order the
+    // slot's MMA warp consumes them).
     const int s = warp == kPpProducer1;
     Cursor cu;
     pp_cursor_init(a, cu, s, T, G);
@@ -820,9 +833,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         cu.bh * a.Np + cu.qb * TILE, &c->q_full[s], pol_q);
         ++qf;
       }
-      const int row = cu.bh * a.Npk + cursor_kb(a, cu) * BK;
-      // the step's second block (the first again when the count is odd)
-      const int row2 = (L::PAIR == 2 && cu.j + 1 < cu.n) ? cu.bh * a.Npk + cursor_kb_at(a, cu, cu.j + 1) * BK : row;
+      // first key row of each piece of the step (past the walk's end: the last
+      // real piece again, masked by the softmax)
+      int prow[L::PPS];
+      const int np = cu.n * L::PPB;
+#pragma unroll
+      for (int p = 0; p < L::PPS; ++p) {
+        const int gp = min(cu.j + p, np - 1);
+        prow[p] = cu.bh * a.Npk + cursor_kb_at(a, cu, gp / L::PPB) * BK + (gp % L::PPB) * L::PK;
+      }
 #pragma unroll 1
       for (int kv = 0; kv < 2; ++kv) {
         const int e = g % R;
@@ -831,15 +850,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx_w(&c->ring_full[s][e], L::STEP_BYTES);
         const CUtensorMap* tm = kv ? &tmV : &tmK;
 #pragma unroll
-        for (int x = 0; x < D / 64; ++x) {
-          tma_load_2d_w(ring + e * L::STEP_BYTES + x * L::SBOX_BYTES, tm, x * 64, row, &c->ring_full[s][e], pol);
-          if constexpr (L::PAIR == 2)
-            tma_load_2d_w(ring + e * L::STEP_BYTES + x * L::SBOX_BYTES + L::KBOX_BYTES, tm, x * 64, row2,
+        for (int x = 0; x < D / 64; ++x)
+#pragma unroll
+          for (int p = 0; p < L::PPS; ++p)
+            tma_load_2d_w(ring + e * L::STEP_BYTES + x * L::SBOX_BYTES + p * L::PBOX_BYTES, tm, x * 64, prow[p],
                           &c->ring_full[s][e], pol);
-        }
         ++g;
       }
-      cursor_step(a, cu, T, 2 * G, L::PAIR);
+      cursor_step(a, cu, T, 2 * G, L::PPS, L::PPB);
     }
     if (lane == 0) {
       if (!ok) {
@@ -903,7 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit_w(&c->s_full[s]);
       mma_commit_w(&c->ring_empty[s][e]);
       if (cu.j == 0) ++qt;
-      if (cu.j + L::PAIR >= cu.n) mma_commit_w(&c->q_empty[s]);
+      if (cu.j + L::PPS >= cu.n * L::PPB) mma_commit_w(&c->q_empty[s]);
       ++g;
       return true;
     };
@@ -930,10 +948,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit_w(&c->ring_empty[s][e]);
       if (cu.j == 0) ++ot;
-      if (cu.j + L::PAIR >= cu.n) mma_commit_w(&c->o_full[s]);
+      if (cu.j + L::PPS >= cu.n * L::PPB) mma_commit_w(&c->o_full[s]);
       ++g;
       ++gb;
-      cursor_step(a, cu, T, 2 * G, L::PAIR);
+      cursor_step(a, cu, T, 2 * G, L::PPS, L::PPB);
       return cu.done ? true : issue_s(s_c);
     };
     bool due0 = false, due1 = false;   // an S was issued whose PV is outstanding
@@ -1004,7 +1022,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       float s_best = -INFINITY;   // largest raw score of the row (normalisation fix-up)
       constexpr int SK = L::SK;
-      for (int j = 0; j < tl.n; j += L::PAIR, ++gb) {
+      const int np = tl.n * L::PPB;   // pieces of this tile's walk
+      for (int j = 0; j < np; j += L::PPS, ++gb) {
         const bool got = mbar_wait(&c->s_full[slot], gb & 1, &c->abort, a.spin_ns);
         ok = __all_sync(0xffffffffu, got);
         if (!ok) break;
@@ -1017,19 +1036,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (SK % 32 == 16) tmem_ld16(t_s + SK / 32 * 32, *reinterpret_cast<uint32_t(*)[16]>(&r[SK / 32 * 32]));
         tmem_ld_wait();
         reg_fence(r);
-        // Key columns past the sequence end exist only in the highest kept
-        // block; with two blocks per step, a step of one block masks its
-        // second half (the first block repeated) entirely.
-        int lim0 = BK, lim1 = BK;
-        if (j == j_last) lim0 = valid_last;
-        if constexpr (L::PAIR == 2) {
-          if (j + 1 >= tl.n) lim1 = 0;
-          else if (j + 1 == j_last) lim1 = valid_last;
+        // Valid keys of each piece: key columns past the sequence end exist
+        // only in the highest kept block; pieces past the walk's end (the last
+        // real piece repeated) are masked entirely.
+        int lim[L::PPS];
+        bool partial = false;
+#pragma unroll
+        for (int p = 0; p < L::PPS; ++p) {
+          const int gp = j + p;
+          lim[p] = gp >= np ? 0
+                 : gp / L::PPB == j_last ? max(0, min(L::PK, valid_last - (gp % L::PPB) * L::PK))
+                                         : L::PK;
+          partial |= lim[p] < L::PK;
         }
-        if (lim0 < BK || lim1 < BK) {
+        if (partial) {
 #pragma unroll
           for (int i = 0; i < SK; ++i)
-            if (i < BK ? i >= lim0 : i - BK >= lim1) r[i] = f2u(-INFINITY);
+            if (i % L::PK >= lim[i / L::PK]) r[i] = f2u(-INFINITY);
         }
         float mx0 = u2f(r[0]), mx1 = u2f(r[1]), mx2 = u2f(r[2]), mx3 = u2f(r[3]);
 #pragma unroll
@@ -1174,7 +1197,7 @@ std::atomic<int> g_num_sms[kMaxDevices];
 // 144-key blocks); there the kernel that splits each block's keys between two
 // warps of the same rows.
 template <int D, int BK>
-constexpr bool kUsePp = (BK <= 128 ? 128 : 160) + D <= 256;
+constexpr bool kUsePp = ((cgcd(BK, TILE) >= 32 ? TILE : BK) <= 128 ? 128 : 160) + D <= 256;
 
 template <int D, int BK>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TcArgs& a,
@@ -1235,8 +1258,12 @@ int launch_tc_fwd(const void* q, const void* k, const void* v, int d, const TcAr
   const uint32_t bk = static_cast<uint32_t>(a.block_k);
   int rc;
   if ((rc = make_tmap_bf16(&tq, q, qrows, d, TILE)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tk, k, krows, d, bk)) != CALIBATT_OK) return rc;
-  if ((rc = make_tmap_bf16(&tv, v, krows, d, bk)) != CALIBATT_OK) return rc;
+  // K and V are copied in pieces of gcd(bk, 128) rows where that is at least
+  // 32 (two-slot kernel, 128-key steps), else in whole blocks
+  const int pg = cgcd(static_cast<int>(bk), TILE);
+  const uint32_t box = pg >= 32 ? static_cast<uint32_t>(pg) : bk;
+  if ((rc = make_tmap_bf16(&tk, k, krows, d, box)) != CALIBATT_OK) return rc;
+  if ((rc = make_tmap_bf16(&tv, v, krows, d, box)) != CALIBATT_OK) return rc;
   switch (bk) {
     case 64: return d == 128 ? launch_fwd<128, 64>(tq, tk, tv, a, s) : launch_fwd<64, 64>(tq, tk, tv, a, s);
     case 80: return d == 128 ? launch_fwd<128, 80>(tq, tk, tv, a, s) : launch_fwd<64, 80>(tq, tk, tv, a, s);
