@@ -678,13 +678,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // TMEM loads, stores and waits overlap the other slot's exponentials.
 //
 // TMEM (512 columns): slot s owns [256 s, 256 s + 256): S_s at
-// [256 s, 256 s + BK) and O_s at [256 s + OC, 256 s + OC + D) with OC = 128
-// (160 for BK = 144).  P overwrites the first BK / 2 columns of S_s as bf16
-// pairs: the A operand of the PV MMA.  With one score buffer per slot the
-// order per slot is S(j), softmax(j), PV(j), S(j + 1): S(j + 1) may overwrite
-// P(j) because the in-order tensor pipe has consumed it, and the commit that
-// signals S(j + 1) also covers PV(j), so O_s can be rescaled as soon as the
-// scores of block j + 1 are visible.
+// [256 s, 256 s + SK) and O_s at [256 s + OC, 256 s + OC + D), where a step
+// holds SK keys (128 for BK = 64, 96, 128; the block for 80 and 144) and
+// OC = 128 (160 for SK = 144).  P overwrites the first SK / 2 columns of S_s
+// as bf16 pairs: the A operand of the PV MMA.  With one score buffer per slot
+// the order per slot is S(j), softmax(j), PV(j), S(j + 1): S(j + 1) may
+// overwrite P(j) because the in-order tensor pipe has consumed it, and the
+// commit that signals S(j + 1) also covers PV(j), so O_s can be rescaled as
+// soon as the scores of step j + 1 are visible.
 // ===========================================================================
 
 constexpr int cgcd(int x, int y) { return y == 0 ? x : cgcd(y, x % y); }
