@@ -153,3 +153,41 @@ def test_main_refuses_a_world_size_other_than_gpus(monkeypatch):
     monkeypatch.setattr(bench.sys, "argv", ["bench.py", "--gpus", "4"])
     with pytest.raises(SystemExit, match="WORLD_SIZE=2"):
         bench.main()
+
+
+def test_clock_sampler_keeps_the_timed_window(tmp_path):
+    # nvidia-smi rows (timestamped) before, inside and after the timed region:
+    # only the rows inside it count; a region shorter than the sampling period
+    # falls back to the samples nearest to it.
+    from datetime import datetime
+
+    def fake_rows(cs, now, offsets, clocks, cap):
+        lines = []
+        for dt, mhz in zip(offsets, clocks):
+            ts = datetime.fromtimestamp(now + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            lines.append(f"{ts}, 0, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, {cap}")
+        cs.path.write_text("\n".join(lines) + "\n")
+
+    class Proc:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            pass
+
+    now = 1_800_000_000.0
+    cs = bench.ClockSampler(0)
+    cs.path = tmp_path / "clocks.csv"
+    fake_rows(cs, now, (-1.0, 0.02, 0.04, 1.0), (1200, 1800, 1810, 1300), "Active")
+    cs.proc, cs.fh = Proc(), open(os.devnull, "w")
+    cs.mark_window(now, now + 0.05)
+    rec = cs.stop()
+    assert rec["samples"] == 2 and rec["sm_mhz"] == 1805.0 and rec["reasons"] == ["sw_power_cap"]
+
+    cs = bench.ClockSampler(0)
+    cs.path = tmp_path / "clocks2.csv"
+    fake_rows(cs, now, (-0.2, -0.03, 0.5), (1500, 1900, 1600), "Not Active")
+    cs.proc, cs.fh = Proc(), open(os.devnull, "w")
+    cs.mark_window(now, now + 0.01)
+    rec = cs.stop()
+    assert rec["samples"] == 2 and rec["sm_mhz"] == 1700.0 and rec["reasons"] == []
