@@ -60,6 +60,22 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _check_buf(name, t, shape, dtype):
+    """Raises unless the caller-supplied buffer ``t`` (None: not given) has
+    exactly ``shape`` and ``dtype``.  The library reads or writes that many
+    elements through the bare pointer and cannot check the size itself."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(int(x) for x in shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} of shape {tuple(int(x) for x in shape)}, "
+                         f"got {t.dtype} of shape {tuple(t.shape)}")
+
+
+def _check_status(status):
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status must be an int32 tensor with at least one element")
+
+
 def default_scale(d):
     """float32 of 1/sqrt(d): the softmax scale the kernels multiply by."""
     return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
@@ -147,10 +163,13 @@ def sparse_attn_fwd(q, k, v, bl: BlockList, N, scale=None, map_offset=0, return_
     Returns O (and LSE [B, H, Np] fp32 when ``return_lse``).  ``status`` is an
     optional int32 CUDA tensor that receives device-side error codes.
     """
-    _need_cuda(q, k, v)
     B, H, Np, d = q.shape
     if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share shape and dtype")
+    _check_buf("out", out, q.shape, q.dtype)
+    _check_buf("lse", lse, (B, H, Np), torch.float32)
+    _check_status(status)
+    _need_cuda(q, k, v)
     scale = default_scale(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
@@ -174,11 +193,14 @@ def sparse_attn_fwd_qk(q, k, v, bl: BlockList, Nq, Nk, scale=None, map_offset=0,
     key padding follows the key-block size (any of 64, 80, 96, 128, 144)
     independently of the query blocks.  Returns O [B, H, Npq, d] (and LSE).
     """
-    _need_cuda(q, k, v)
     B, H, Npq, d = q.shape
     Npk = k.shape[2]
     if k.shape != (B, H, Npk, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("k, v must be [B, H, Npk, d] of q's dtype")
+    _check_buf("out", out, q.shape, q.dtype)
+    _check_buf("lse", lse, (B, H, Npq), torch.float32)
+    _check_status(status)
+    _need_cuda(q, k, v)
     scale = default_scale(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty_like(q)
@@ -220,10 +242,14 @@ def sparse_attn_fwd_streamed(q, k, v, bl: BlockList, N, staging, scale=None, map
     lse_d = staging[4] if len(staging) > 4 else None
     if (lse is None) != (lse_d is None):
         raise ValueError("pass lse together with an lse staging buffer")
-    _need_cuda(qd, kd, vd, od, lse_d, status)
     for t in (qd, kd, vd, od):
         if t.shape != q.shape or t.dtype != q.dtype:
             raise ValueError("staging buffers must match q's shape and dtype")
+    _check_buf("out", out, q.shape, q.dtype)
+    _check_buf("lse", lse, (B, H, Np), torch.float32)
+    _check_buf("lse staging buffer", lse_d, (B, H, Np), torch.float32)
+    _check_status(status)
+    _need_cuda(qd, kd, vd, od, lse_d, status)
     scale = default_scale(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
@@ -326,8 +352,11 @@ def spatial_similarity(q, k, N, frames, rows, cols, scale=None, status=None):
     column): near 1 for maps that repeat across spatial rows (paper page,
     Figure 4, Figure 6(a), Figure S13).
     """
-    _need_cuda(q, k)
     H, Np, d = q.shape
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must share shape and dtype")
+    _check_status(status)
+    _need_cuda(q, k)
     scale = default_scale(d) if scale is None else float(scale)
     n = ctypes.c_size_t(0)
     check(load().calibatt_spatial_similarity_workspace_size(H, Np, ctypes.byref(n)))
@@ -335,7 +364,7 @@ def spatial_similarity(q, k, N, frames, rows, cols, scale=None, status=None):
     out = torch.empty(H, dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
         check(load().calibatt_spatial_similarity(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), int(frames),
-                                                 int(rows), int(cols), scale, _ptr(out), _ptr(ws), ws.numel(),
+                                                 int(rows), int(cols), scale, _ptr(out), _ptr(ws), ws.nbytes,
                                                  _ptr(status), _stream(q.device)))
     return out
 
@@ -344,6 +373,8 @@ def repetition_flags(scores, tau=0.87):
     """Repetition dictionary (``calibatt_repetition_flags``): from per-input
     scores [n_inputs, n_maps] float32 (CUDA), the mean score per map and the
     flags mean >= tau (paper page, Figure 5(a), Figure S13: tau = 0.87)."""
+    if scores.dim() != 2 or scores.dtype != torch.float32:
+        raise ValueError("scores must be float32 [n_inputs, n_maps]")
     _need_cuda(scores)
     n_inputs, n_maps = scores.shape
     mean = torch.empty(n_maps, dtype=torch.float32, device=scores.device)
@@ -362,14 +393,17 @@ def _calib_workspace(H, N, Np, d, bq, bk, device):
 
 def block_energy(q, k, N, block_q=128, block_k=128, scale=None, status=None, workspace=None):
     """Block energies [H, nqb, nkb] fp32 of one input; q, k: [H, Np, d]."""
-    _need_cuda(q, k)
     H, Np, d = q.shape
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must share shape and dtype")
+    _check_status(status)
+    _need_cuda(q, k, workspace)
     scale = default_scale(d) if scale is None else float(scale)
     E = torch.empty((H, Np // block_q, -(-int(N) // block_k)), device=q.device, dtype=torch.float32)
     ws = _calib_workspace(H, N, Np, d, block_q, block_k, q.device) if workspace is None else workspace
     with torch.cuda.device(q.device):
         check(load().calibatt_block_energy(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q, block_k,
-                                           scale, _ptr(E), _ptr(ws), ws.numel(), _ptr(status), _stream(q.device)))
+                                           scale, _ptr(E), _ptr(ws), ws.nbytes, _ptr(status), _stream(q.device)))
     return E
 
 
@@ -382,10 +416,15 @@ def block_energy_noalloc(q, k, N, block_q=128, block_k=128, scale=None, status=N
     Pass ``out`` ([H, nqb, nkb] float32) to avoid the one allocation this
     wrapper would otherwise make for the result.
     """
-    _need_cuda(q, k)
     H, Np, d = q.shape
+    if k.shape != q.shape or k.dtype != q.dtype:
+        raise ValueError("q and k must share shape and dtype")
+    eshape = (H, Np // block_q, -(-int(N) // block_k))
+    _check_buf("out", out, eshape, torch.float32)
+    _check_status(status)
+    _need_cuda(q, k)
     scale = default_scale(d) if scale is None else float(scale)
-    E = torch.empty((H, Np // block_q, -(-int(N) // block_k)), device=q.device, dtype=torch.float32) if out is None else out
+    E = torch.empty(eshape, device=q.device, dtype=torch.float32) if out is None else out
     _need_cuda(E, status)
     with torch.cuda.device(q.device):
         check(load().calibatt_block_energy_noalloc(_ptr(q), _ptr(k), H, int(N), Np, d, _dtype_code(q), block_q,
@@ -395,8 +434,12 @@ def block_energy_noalloc(q, k, N, block_q=128, block_k=128, scale=None, status=N
 
 def select_vote(energy, mode, param, votes, energy_sum):
     """Adds one input's selection (top-k fraction or energy eps) into votes / energy_sum (in place)."""
-    _need_cuda(energy, votes, energy_sum)
+    if energy.dim() != 3 or energy.dtype != torch.float32:
+        raise ValueError("energy must be float32 [H, nqb, nkb]")
     H, nqb, nkb = energy.shape
+    _check_buf("votes", votes, energy.shape, torch.int32)
+    _check_buf("energy_sum", energy_sum, energy.shape, torch.float32)
+    _need_cuda(energy, votes, energy_sum)
     with torch.cuda.device(energy.device):
         check(load().calibatt_select_vote(_ptr(energy), H, nqb, nkb, int(mode), float(param), _ptr(votes),
                                           _ptr(energy_sum), _stream(energy.device)))
@@ -405,6 +448,9 @@ def select_vote(energy, mode, param, votes, energy_sum):
 
 def finalize_mask(votes, energy_sum, min_votes):
     """uint8 mask [H, nqb, nkb] = votes >= min_votes, with the empty-row guard."""
+    if votes.dim() != 3 or votes.dtype != torch.int32:
+        raise ValueError("votes must be int32 [H, nqb, nkb]")
+    _check_buf("energy_sum", energy_sum, votes.shape, torch.float32)
     _need_cuda(votes, energy_sum)
     H, nqb, nkb = votes.shape
     mask = torch.empty((H, nqb, nkb), dtype=torch.uint8, device=votes.device)
@@ -425,10 +471,16 @@ def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mo
     n = len(q_list)
     if n != len(k_list) or n == 0:
         raise ValueError("need the same non-zero number of q and k tensors")
-    _need_cuda(*q_list, *k_list)
     H, Np, d = q_list[0].shape
+    for t in (*q_list, *k_list):
+        if t.shape != q_list[0].shape or t.dtype != q_list[0].dtype or t.device != q_list[0].device:
+            raise ValueError("every q and k must share shape, dtype and device")
     dev = q_list[0].device
     nqb, nkb = Np // block_q, -(-int(N) // block_k)
+    _check_buf("votes", votes, (H, nqb, nkb), torch.int32)
+    _check_buf("energy_sum", energy_sum, (H, nqb, nkb), torch.float32)
+    _check_status(status)
+    _need_cuda(*q_list, *k_list, votes, energy_sum)
     scale = default_scale(d) if scale is None else float(scale)
     if votes is None:
         votes = torch.zeros((H, nqb, nkb), dtype=torch.int32, device=dev)
@@ -443,7 +495,7 @@ def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mo
     with torch.cuda.device(dev):
         check(load().calibatt_calibrate(qp, kp, n, H, int(N), Np, d, _dtype_code(q_list[0]), block_q, block_k, scale,
                                         int(select_mode), float(select_param), _ptr(votes), _ptr(energy_sum),
-                                        int(min_votes), _ptr(mask), _ptr(ws), ws.numel(), _ptr(status),
+                                        int(min_votes), _ptr(mask), _ptr(ws), ws.nbytes, _ptr(status),
                                         _stream(dev)))
     return mask, votes, energy_sum
 
@@ -472,8 +524,12 @@ def timestep_clusters(masks, tau):
 
 def share_masks(masks, run_of, n_runs):
     """Union masks [n_runs, H, nqb, nkb] uint8 of the runs ``run_of`` ([L, T] int32)."""
-    _need_cuda(masks)
+    if masks.dtype != torch.uint8 or masks.dim() != 5:
+        raise ValueError("masks must be uint8 [L, T, H, nqb, nkb]")
     L, T, H, nqb, nkb = masks.shape
+    if tuple(run_of.shape) != (L, T):
+        raise ValueError(f"run_of must have shape {(L, T)}, got {tuple(run_of.shape)}")
+    _need_cuda(masks)
     run_dev = run_of.to(device=masks.device, dtype=torch.int32).contiguous()
     shared = torch.empty((int(n_runs), H, nqb, nkb), dtype=torch.uint8, device=masks.device)
     with torch.cuda.device(masks.device):
@@ -496,6 +552,8 @@ def share_timesteps(masks, tau):
 
 def interval_counts(masks):
     """int32 [n_maps, nqb]: kept-block intervals of every row of uint8 masks [n_maps, nqb, nkb]."""
+    if masks.dtype != torch.uint8 or masks.dim() != 3:
+        raise ValueError("masks must be uint8 [n_maps, nqb, nkb]")
     _need_cuda(masks)
     n_maps, nqb, nkb = masks.shape
     counts = torch.empty((n_maps, nqb), dtype=torch.int32, device=masks.device)
@@ -508,8 +566,12 @@ def merge_intervals(masks, width_per_map):
     """Merges, in place, every row of map i to at most width_per_map[i] intervals.
 
     Returns the number of filled blocks (synchronizes)."""
-    _need_cuda(masks)
+    if masks.dtype != torch.uint8 or masks.dim() != 3:
+        raise ValueError("masks must be uint8 [n_maps, nqb, nkb]")
     n_maps, nqb, nkb = masks.shape
+    if torch.as_tensor(width_per_map).numel() != n_maps:
+        raise ValueError(f"width_per_map must have one entry per map ({n_maps})")
+    _need_cuda(masks)
     width = torch.as_tensor(width_per_map, dtype=torch.int32).to(masks.device).contiguous()
     filled = torch.zeros(1, dtype=torch.int64, device=masks.device)
     with torch.cuda.device(masks.device):
@@ -608,22 +670,24 @@ def _compile_ws(n_maps, nqb, nkb, dev):
 
 def compile_size(masks, dedup=DEDUP_HASH, workspace=None):
     """(nnz, n_pat, nnz_pat) of compiling ``masks`` [n_maps, nqb, nkb] uint8 (synchronizes)."""
-    _need_cuda(masks)
+    if masks.dtype != torch.uint8 or masks.dim() != 3:
+        raise ValueError("masks must be uint8 [n_maps, nqb, nkb]")
+    _need_cuda(masks, workspace)
     n_maps, nqb, nkb = masks.shape
     ws = _compile_ws(n_maps, nqb, nkb, masks.device) if workspace is None else workspace
     nnz, n_pat, nnz_pat = ctypes.c_int64(0), ctypes.c_int32(0), ctypes.c_int32(0)
     with torch.cuda.device(masks.device):
         check(load().calibatt_compile_size(_ptr(masks), n_maps, nqb, nkb, int(dedup), ctypes.byref(nnz),
-                                           ctypes.byref(n_pat), ctypes.byref(nnz_pat), _ptr(ws), ws.numel(),
+                                           ctypes.byref(n_pat), ctypes.byref(nnz_pat), _ptr(ws), ws.nbytes,
                                            _stream(masks.device)))
     return nnz.value, n_pat.value, nnz_pat.value
 
 
 def compile(masks, block_q=128, block_k=128, dedup=DEDUP_HASH, with_csr=True):
     """Compiles uint8 masks [n_maps, nqb, nkb] into a :class:`BlockList` (synchronizes)."""
+    if masks.dtype != torch.uint8 or masks.dim() != 3:
+        raise TypeError("masks must be uint8 [n_maps, nqb, nkb]")
     _need_cuda(masks)
-    if masks.dtype != torch.uint8:
-        raise TypeError("masks must be uint8")
     n_maps, nqb, nkb = masks.shape
     dev = masks.device
     ws = _compile_ws(n_maps, nqb, nkb, dev)
@@ -644,7 +708,7 @@ def compile(masks, block_q=128, block_k=128, dedup=DEDUP_HASH, with_csr=True):
         s.pat_off = None
     with torch.cuda.device(dev):
         check(load().calibatt_compile(_ptr(masks), n_maps, nqb, nkb, int(dedup), block_q, block_k, ctypes.byref(s),
-                                      _ptr(ws), ws.numel(), _stream(dev)))
+                                      _ptr(ws), ws.nbytes, _stream(dev)))
     return bl
 
 

@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_and_weak_scaling_gloo():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     for rank in range(world):
@@ -88,7 +88,7 @@ def test_sharded_calibration_gathers_inputs_in_global_order_gloo(world):
     # every input's energies in global input order (rank-major), whatever the
     # per-rank counts, so that selection, votes and the float32 energy sums
     # replay the single-GPU order exactly.
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_gather_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     n = sum([2, 1, 3][:world])
