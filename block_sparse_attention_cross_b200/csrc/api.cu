@@ -460,6 +460,7 @@ int calibatt_select_vote(const float* energy, int H, int nqb, int nkb, int selec
     return set_error(CALIBATT_E_INVALID, "energy, votes and energy_sum must be non-NULL");
   if (H <= 0 || nqb <= 0 || nkb <= 0) return set_error(CALIBATT_E_INVALID, "bad sizes");
   if (nkb > 2048) return set_error(CALIBATT_E_UNSUPPORTED, "at most 2048 key blocks per row");
+  if (static_cast<long long>(H) * nqb >= (1ll << 31)) return set_error(CALIBATT_E_UNSUPPORTED, "H*nqb too large");
   int topk = 0;
   double eps = 0.0;
   if (select_mode == CALIBATT_SELECT_TOPK) {
@@ -480,6 +481,7 @@ int calibatt_finalize_mask(const int32_t* votes, const float* energy_sum, int H,
   if (votes == nullptr || energy_sum == nullptr || mask_out == nullptr)
     return set_error(CALIBATT_E_INVALID, "votes, energy_sum and mask must be non-NULL");
   if (H <= 0 || nqb <= 0 || nkb <= 0) return set_error(CALIBATT_E_INVALID, "bad sizes");
+  if (static_cast<long long>(H) * nqb >= (1ll << 31)) return set_error(CALIBATT_E_UNSUPPORTED, "H*nqb too large");
   if (min_votes < 0) return set_error(CALIBATT_E_INVALID, "min_votes must be >= 0");
   return launch_finalize(votes, energy_sum, H * nqb, nkb, min_votes, mask_out,
                          reinterpret_cast<cudaStream_t>(stream));

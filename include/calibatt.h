@@ -336,6 +336,10 @@ int calibatt_calibrate_workspace_size(int H, int N, int Np, int d, int block_q, 
  * (float32).
  *  energy      [H, nqb, nkb] float32 (read);  votes_inout int32, energy_sum_inout
  *              float32, both [H, nqb, nkb] (read-modify-write).
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, a non-positive size, an
+ * unknown mode or a parameter out of range (frac in (0, 1], eps in [0, 1));
+ * CALIBATT_E_UNSUPPORTED for nkb > 2048 or H * nqb >= 2^31.  Asynchronous on
+ * `stream`; nothing is enqueued for a rejected call.
  */
 int calibatt_select_vote(const float* energy, int H, int nqb, int nkb, int select_mode,
                          double select_param, int32_t* votes_inout, float* energy_sum_inout,
@@ -345,7 +349,11 @@ int calibatt_select_vote(const float* energy, int H, int nqb, int nkb, int selec
  * calibatt_finalize_mask -- agreement threshold (paper page, Figure 7, rho).
  * mask = votes >= min_votes.  A row left empty keeps exactly one key block:
  * the one with the most votes, then the largest energy_sum, then the
- * smallest index.  mask_out [H, nqb, nkb] uint8 (0/1).
+ * smallest index.  votes int32 and energy_sum float32 [H, nqb, nkb] (read);
+ * mask_out [H, nqb, nkb] uint8 (0/1).
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, a non-positive size or
+ * min_votes < 0; CALIBATT_E_UNSUPPORTED for H * nqb >= 2^31.  Asynchronous on
+ * `stream`; nothing is enqueued for a rejected call.
  */
 int calibatt_finalize_mask(const int32_t* votes, const float* energy_sum, int H, int nqb, int nkb,
                            int min_votes, uint8_t* mask_out, calibatt_stream_t stream);

@@ -152,6 +152,10 @@ def test_calibration_and_compile_validation(lib):
     assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_TOPK, 0.0, fake, fake, None) == _lib.E_INVALID
     assert lib.calibatt_select_vote(fake, 2, 8, 8, _lib.SELECT_ENERGY, 1.0, fake, fake, None) == _lib.E_INVALID
     assert lib.calibatt_finalize_mask(fake, fake, 2, 8, 8, -1, fake, None) == _lib.E_INVALID
+    # H * nqb rows at 2^31 would overflow the row index: refused before any launch
+    assert lib.calibatt_select_vote(fake, 65536, 32768, 8, _lib.SELECT_TOPK, 0.25, fake, fake, None) == \
+        _lib.E_UNSUPPORTED
+    assert lib.calibatt_finalize_mask(fake, fake, 65536, 32768, 8, 1, fake, None) == _lib.E_UNSUPPORTED
     nnz, npat, nnzp = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
     assert lib.calibatt_compile_size(fake, 1, 8, 40000, 1, ctypes.byref(nnz), ctypes.byref(npat), ctypes.byref(nnzp),
                                      fake, 1 << 20, None) == _lib.E_UNSUPPORTED
