@@ -35,6 +35,8 @@ __all__ = [
     "compile", "compile_size", "selftest_wait_timeout", "min_votes_for", "topk_count", "launch_count",
     "default_scale", "CalibattError", "BF16", "FP32", "SELECT_TOPK", "SELECT_ENERGY",
     "DEDUP_NONE", "DEDUP_HASH", "DEDUP_HASH_WEAK", "load",
+    "save_state", "load_state", "save_calibration", "load_calibration", "save_masks", "load_masks",
+    "save_blocklist", "load_blocklist",
 ]
 
 
@@ -461,16 +463,20 @@ def finalize_mask(votes, energy_sum, min_votes):
 
 
 def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mode=SELECT_TOPK, select_param=0.25,
-              rho=0.5, min_votes=None, votes=None, energy_sum=None, finalize=True, status=None):
+              rho=0.5, min_votes=None, votes=None, energy_sum=None, finalize=True, status=None, inputs_before=0):
     """Calibration pass.  Returns (mask or None, votes, energy_sum).
 
     ``votes`` / ``energy_sum`` (int32 / fp32 [H, nqb, nkb]) accumulate across
-    calls, so calibration can resume; ``min_votes`` defaults to
-    ceil(rho * total inputs seen), the total taken from ``votes``' callers.
+    calls, so calibration can resume: pass the state after ``inputs_before``
+    earlier inputs (see :mod:`.dictionary` for saving it).  ``min_votes``
+    defaults to ceil(rho * I) with I = inputs_before + len(q_list), the total
+    number of inputs behind the votes.
     """
     n = len(q_list)
     if n != len(k_list) or n == 0:
         raise ValueError("need the same non-zero number of q and k tensors")
+    if int(inputs_before) < 0 or (int(inputs_before) > 0 and (votes is None or energy_sum is None)):
+        raise ValueError("inputs_before > 0 needs the votes and energy_sum of those inputs")
     H, Np, d = q_list[0].shape
     for t in (*q_list, *k_list):
         if t.shape != q_list[0].shape or t.dtype != q_list[0].dtype or t.device != q_list[0].device:
@@ -487,7 +493,7 @@ def calibrate(q_list, k_list, N, block_q=128, block_k=128, scale=None, select_mo
     if energy_sum is None:
         energy_sum = torch.zeros((H, nqb, nkb), dtype=torch.float32, device=dev)
     if min_votes is None:
-        min_votes = min_votes_for(rho, n)
+        min_votes = min_votes_for(rho, int(inputs_before) + n)
     mask = torch.empty((H, nqb, nkb), dtype=torch.uint8, device=dev) if finalize else None
     ws = _calib_workspace(H, N, Np, d, block_q, block_k, dev)
     qp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in q_list])
@@ -719,3 +725,7 @@ def selftest_wait_timeout(limit_ns=10_000_000, device=None):
     with torch.cuda.device(dev):
         check(load().calibatt_selftest_wait_timeout(int(limit_ns), _ptr(status), _stream(dev)))
     return int(status.item())
+
+
+from .dictionary import (load_blocklist, load_calibration, load_masks, load_state, save_blocklist,  # noqa: E402
+                         save_calibration, save_masks, save_state)

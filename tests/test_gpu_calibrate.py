@@ -147,6 +147,30 @@ def near_tie_rows(E, k):
     return gap < 1e-4 * s[..., 0]
 
 
+def test_calibration_resumes_from_saved_state(tmp_path):
+    # Votes and energy sums add up over inputs (Figure 3(b): a block's count
+    # over the calibration prompts): a calibration saved after 3 of 6 inputs,
+    # reloaded and continued with the other 3 (inputs_before = 3), ends with
+    # the votes, energy sums and mask of one 6-input pass, bit for bit.  The
+    # threshold counts all 6 inputs: ceil(0.5 * 6) = 3 votes, not 2.
+    H, I = 2, 6
+    w, inputs = small_inputs(I, H, syn.VideoGrid(2, 20, 50), 128, seed_base=50)
+    qd = [bf16_pair(q)[1] for q, _ in inputs]
+    kd = [bf16_pair(k)[1] for _, k in inputs]
+    mask1, votes1, esum1 = cba.calibrate(qd, kd, w.N, select_param=0.3, rho=0.5)
+    m_half, v_half, e_half = cba.calibrate(qd[:3], kd[:3], w.N, select_param=0.3, rho=0.5, finalize=False)
+    assert m_half is None
+    p = tmp_path / "calib.npz"
+    cba.save_calibration(p, v_half, e_half, 3, select_param=0.3, rho=0.5)
+    v, e, n, meta = cba.load_calibration(p, device="cuda")
+    mask2, votes2, esum2 = cba.calibrate(qd[3:], kd[3:], w.N, select_param=meta["select_param"], rho=meta["rho"],
+                                         votes=v, energy_sum=e, inputs_before=n)
+    assert torch.equal(votes2, votes1)
+    assert torch.equal(esum2, esum1)
+    assert torch.equal(mask2, mask1)
+    assert torch.equal(mask1, cba.finalize_mask(votes1, esum1, 3))
+
+
 def test_calibrate_small_end_to_end():
     H, I = 2, 4
     w, inputs = small_inputs(I, H, syn.VideoGrid(3, 30, 52), 128)
