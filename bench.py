@@ -405,6 +405,16 @@ def workload_label(name, w, bl):
             f"d={w.d}, bf16, {blocks}, {100 * bl.density:.1f}% of blocks kept (structured mask)")
 
 
+def linear_fit(x, y):
+    """Least-squares line y = slope * x + intercept and its R^2 (1 when y is constant)."""
+    x = np.asarray(x, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    slope, intercept = np.polyfit(x, y, 1)
+    ss = float(np.sum((y - y.mean()) ** 2))
+    r2 = 1.0 - float(np.sum((y - (slope * x + intercept)) ** 2)) / ss if ss > 0 else 1.0
+    return float(slope), float(intercept), r2
+
+
 def time_calls(fn, steps, warmup, torch, dist=None):
     for _ in range(warmup):
         fn()
@@ -503,6 +513,17 @@ def _sweep_workload(device, pk):
     tot, _ = time_calls(step, 2, 1, torch)
     ms = tot / 2
     kept = kept_flops(bl.nnz, w.d, w.B) / (ms / 1e3) / 1e12
+    # per-call device time (one timed step per call, in dictionary order)
+    # against the call's density: the kept fraction of its H maps
+    done = [0]
+
+    def one_call():
+        cba.sparse_attn_fwd(q, k, v, bl, w.N, map_offset=offsets[done[0] % len(offsets)], out=out)
+        done[0] += 1
+
+    _, call_ms = time_calls(one_call, len(offsets), 0, torch)
+    call_dens = [float(masks[mo:mo + w.H].mean()) for mo in offsets]
+    c_sl, c_ic, c_r2 = linear_fit(call_dens, call_ms)
     rng = np.random.default_rng(5)
     errs = []
     scale = cba.default_scale(w.d)
@@ -514,6 +535,9 @@ def _sweep_workload(device, pk):
     return {"calls": len(offsets), "maps": int(masks.shape[0]), "mean_density": round(bl.density, 6),
             "ms_per_step": round(ms, 3), "kept_tflops": round(kept, 2),
             "frac_of_bf16_burst": round(kept / pk["bf16_burst"], 4),
+            "per_call_fit": {"ms_per_unit_density": round(c_sl, 4), "intercept_ms": round(c_ic, 4),
+                             "r2": round(c_r2, 5), "density_range": [round(min(call_dens), 4), round(max(call_dens), 4)],
+                             "call_ms_range": [round(min(call_ms), 4), round(max(call_ms), 4)]},
             "parity_sampled": dict(_parity(errs), calls_checked=4, blocks=len(errs))}
 
 
@@ -796,10 +820,7 @@ def main_calibatt(args):
                           "kept_tflops": round(kept_flops(b.nnz, w.d, w.B) / (td / 20 / 1e3) / 1e12, 1)})
         extras["density_sweep"] = dens_sweep
         # wall time against kept fraction: linear fit, and kept-block throughput at 0.2 against 1.0
-        xd = np.asarray([r["density"] for r in dens_sweep])
-        yd = np.asarray([r["ms"] for r in dens_sweep])
-        sl, ic = np.polyfit(xd, yd, 1)
-        r2d = 1.0 - np.sum((yd - (sl * xd + ic)) ** 2) / np.sum((yd - yd.mean()) ** 2)
+        sl, ic, r2d = linear_fit([r["density"] for r in dens_sweep], [r["ms"] for r in dens_sweep])
         def at(d):
             return min(dens_sweep, key=lambda r: abs(r["density"] - d))["kept_tflops"]
         extras["density_fit"] = {"ms_per_unit_density": round(float(sl), 4), "intercept_ms": round(float(ic), 4),

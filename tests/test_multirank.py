@@ -108,6 +108,19 @@ def test_bench_workload_helpers():
     assert bench.workload(8, "sweep").H == 8
 
 
+def test_linear_fit():
+    # an exact line: slope, intercept and R^2 = 1 recovered
+    x = [1.0, 0.8, 0.6, 0.4, 0.25, 0.2, 0.1]
+    sl, ic, r2 = bench.linear_fit(x, [21.5 * d - 0.1 for d in x])
+    assert sl == pytest.approx(21.5) and ic == pytest.approx(-0.1) and r2 == pytest.approx(1.0)
+    # a hand case: y = 1, 0, 3, 2 at x = 0 .. 3 -> slope 0.6, intercept 0.6, residual sum 3.2 of a
+    # total 5, R^2 = 0.36
+    sl, ic, r2 = bench.linear_fit([0, 1, 2, 3], [1, 0, 3, 2])
+    assert sl == pytest.approx(0.6) and ic == pytest.approx(0.6) and r2 == pytest.approx(0.36)
+    # constant y: the line is flat and fits exactly
+    assert bench.linear_fit([0.1, 0.2, 0.3], [2.0, 2.0, 2.0]) == pytest.approx((0.0, 2.0, 1.0))
+
+
 def _replica_probe(path):
     # one replica of the harness on CPU: the torchrun-style environment set by
     # launch_replicas, a gloo group, the max-over-ranks timing and the line
