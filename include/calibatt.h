@@ -17,7 +17,9 @@
  *    *_workspace_size query.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream).  The only calls that synchronize the stream
- *    are calibatt_compile_size and calibatt_compile (they read counts back).
+ *    are those that read results back to the host: calibatt_compile_size,
+ *    calibatt_compile, calibatt_timestep_clusters, calibatt_skiplist_sizes
+ *    and calibatt_blocklist_kept.
  *  - Every call returns a status: CALIBATT_OK (0) or a negative code below.
  *    On a non-zero return nothing was launched unless the code is
  *    CALIBATT_E_CUDA (a launch error).  calibatt_last_error() returns a
@@ -137,6 +139,13 @@ uint64_t calibatt_get_spin_limit_ns(void);
  * key-block sizes); CALIBATT_FP32 with d in {64, 128}, block_q and block_k
  * in {64, 128} (FFMA).  At most 2048 key blocks per row.  Anything else
  * returns CALIBATT_E_UNSUPPORTED.
+ * Errors: CALIBATT_E_INVALID for a NULL or unaligned tensor, a non-positive
+ * size, N > Np, a scale that is not finite and positive, a block list whose
+ * grid does not match Np / block, padding of a whole block or more, or maps
+ * beyond bl->n_maps; CALIBATT_E_UNSUPPORTED as above or for B * H * Np >=
+ * 2^31; CALIBATT_E_CUDA for a launch failure.  On the device a corrupt row
+ * of the block list writes CALIBATT_E_CORRUPT to dev_status (that row's
+ * output becomes 0 / -inf) and a wait that runs out CALIBATT_E_TIMEOUT.
  */
 int calibatt_sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int H, int N, int Np, int d, int dtype, float scale,
@@ -204,6 +213,8 @@ int calibatt_sparse_attn_fwd_qk(const void* q, const void* k, const void* v, voi
  *  src [n_planes, rows_src, row_bytes], dst [n_planes, rows_dst, row_bytes]
  *  (device, 16-byte aligned, row_bytes a multiple of 16); idx [rows_dst]
  *  int32 device.  Asynchronous.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, a non-positive size, a
+ * row_bytes that is not a multiple of 16 or an unaligned src / dst.
  */
 int calibatt_gather_rows(const void* src, void* dst, const int32_t* idx, int n_planes, int rows_src, int rows_dst,
                          int row_bytes, calibatt_stream_t stream);
@@ -368,6 +379,10 @@ int calibatt_finalize_mask(const int32_t* votes, const float* energy_sum, int H,
  *  q_list, k_list  HOST arrays of n_inputs device pointers, each [H, Np, d].
  *  votes_inout, energy_sum_inout, mask_out  [H, Np/block_q, ceil(N/block_k)].
  * Shapes as calibatt_block_energy.
+ * Errors: those of calibatt_block_energy (for every input), of
+ * calibatt_select_vote and, when mask_out is set, of calibatt_finalize_mask;
+ * CALIBATT_E_INVALID for n_inputs < 0 or NULL lists.  All arguments are
+ * checked before the first launch, so a rejected call enqueues nothing.
  */
 int calibatt_calibrate(const void* const* q_list, const void* const* k_list, int n_inputs,
                        int H, int N, int Np, int d, int dtype, int block_q, int block_k,
@@ -390,6 +405,11 @@ int calibatt_calibrate(const void* const* q_list, const void* const* k_list, int
  * calls calibatt_compile, which fills them, writes n_maps .. block_k, and
  * synchronizes; it fails with CALIBATT_E_INVALID if the capacities are
  * smaller than the sizes.  Workspace: calibatt_compile_workspace_size.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, a non-positive size, an
+ * unknown dedup mode or (compile) output capacities below the sizes;
+ * CALIBATT_E_UNSUPPORTED for nkb > 32767, n_maps * nqb >= 2^31 or a pattern
+ * pool beyond int32 indexing; CALIBATT_E_WORKSPACE for a missing or short
+ * workspace; CALIBATT_E_CUDA if a launch or the read-back fails.
  */
 int calibatt_compile_workspace_size(int n_maps, int nqb, int nkb, size_t* bytes);
 int calibatt_compile_size(const uint8_t* masks, int n_maps, int nqb, int nkb, int dedup,
@@ -447,6 +467,9 @@ int calibatt_block_energy_noalloc(const void* q, const void* k, int H, int N, in
  *             256-byte aligned.
  * Synchronizes the stream (the grouping runs on the host from exact integer
  * pair counts computed on the device).  T <= 1024.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, a non-positive size or a NaN
+ * tau; CALIBATT_E_UNSUPPORTED for T > 1024 or L * T > 2^20;
+ * CALIBATT_E_WORKSPACE for a short or unaligned workspace.
  */
 int calibatt_timestep_clusters_workspace_size(int L, int T, int H, size_t* bytes);
 int calibatt_timestep_clusters(const uint8_t* masks, int L, int T, int H, int nqb, int nkb, double tau,
@@ -461,6 +484,9 @@ int calibatt_timestep_clusters(const uint8_t* masks, int L, int T, int H, int nq
  *  shared    [n_runs, H, nqb, nkb] uint8 device (written, 0/1).
  * The call (l, t) then uses map_offset = run_of[l T + t] * H of the shared
  * dictionary.  Asynchronous on `stream`.
+ * Errors: as calibatt_timestep_clusters for the sizes; CALIBATT_E_INVALID for
+ * n_runs outside [1, L * T]; CALIBATT_E_UNSUPPORTED for n_runs * H > 65535.
+ * Run indices in run_of_dev outside [0, n_runs) select no run (harmless).
  */
 int calibatt_share_masks(const uint8_t* masks, int L, int T, int H, int nqb, int nkb, const int32_t* run_of_dev,
                          int n_runs, uint8_t* shared, calibatt_stream_t stream);
@@ -471,6 +497,7 @@ int calibatt_share_masks(const uint8_t* masks, int L, int T, int H, int nqb, int
  * length of the paper page's interval skip lists (Figure S9, Figure S10).
  *  masks   [n_maps, nqb, nkb] uint8 device (nonzero = kept);
  *  counts  [n_maps * nqb] int32 device (written).  Asynchronous.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer or a non-positive size.
  */
 int calibatt_interval_counts(const uint8_t* masks, int n_maps, int nqb, int nkb, int32_t* counts,
                              calibatt_stream_t stream);
@@ -485,6 +512,8 @@ int calibatt_interval_counts(const uint8_t* masks, int n_maps, int nqb, int nkb,
  *  width   [n_maps] int32 device (values below 1 count as 1).
  *  filled  one uint64 on the device: the number of filled blocks is added.
  * Asynchronous.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer or a non-positive size;
+ * CALIBATT_E_UNSUPPORTED for nkb > 2048.
  */
 int calibatt_merge_intervals(uint8_t* masks, int n_maps, int nqb, int nkb, const int32_t* width,
                              unsigned long long* filled, calibatt_stream_t stream);
@@ -527,6 +556,7 @@ int calibatt_skiplist_sizes(const int32_t* counts, int n_maps, int nqb, int nkb,
  * row pointers, int16 columns) and the pattern pool (int32 base and pattern
  * id per row, int32 pattern pointers, int16 offsets); sizes from
  * calibatt_compile_size.  Host arithmetic only.
+ * Errors: CALIBATT_E_INVALID for NULL outputs or sizes out of range.
  */
 int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, int32_t nnz_pat, int64_t* csr_bytes,
                              int64_t* pool_bytes);
@@ -537,6 +567,8 @@ int calibatt_blocklist_bytes(int n_maps, int nqb, int64_t nnz, int32_t n_pat, in
  * of the calibration inputs keep it): min_votes = ceil(rho n_inputs), with
  * rho n_inputs rounded to 9 decimals first (so 0.3 * 10 gives 3), clamped to
  * [0, n_inputs].  Host arithmetic only.
+ * Errors: CALIBATT_E_INVALID for a NULL output, n_inputs <= 0 or a rho that is
+ * not finite.
  */
 int calibatt_min_votes(double rho, int n_inputs, int32_t* min_votes);
 
@@ -544,6 +576,7 @@ int calibatt_min_votes(double rho, int n_inputs, int32_t* min_votes);
  * calibatt_topk_count -- key blocks kept per query-block row by the top-k
  * selection (paper page, Figure 5(a)): ceil(frac nkb) clamped to [1, nkb], the
  * count calibatt_select_vote uses.  Host arithmetic only; frac in (0, 1].
+ * Errors: CALIBATT_E_INVALID for a NULL output, nkb <= 0 or frac outside (0, 1].
  */
 int calibatt_topk_count(double frac, int nkb, int32_t* k);
 
@@ -552,17 +585,20 @@ int calibatt_topk_count(double frac, int nkb, int32_t* k);
  * map_offset + n_maps) of a compiled block list (the sum of their rows'
  * pattern lengths), for per-call density and FLOP counts.  workspace: 8 bytes
  * of device memory (8-byte aligned).  Synchronizes `stream`.
+ * Errors: CALIBATT_E_INVALID for a NULL pointer, maps outside the list or an
+ * unaligned workspace; CALIBATT_E_WORKSPACE for a workspace under 8 bytes;
+ * CALIBATT_E_CUDA if the launch or the read-back fails.
  */
 int calibatt_blocklist_kept(const calibatt_blocklist* bl, int map_offset, int n_maps, int64_t* kept, void* workspace,
                             size_t workspace_bytes, calibatt_stream_t stream);
-
-
 
 /*
  * calibatt_selftest_wait_timeout -- launches one block that waits, with the
  * bounded wait every kernel here uses, on a barrier that nothing completes.
  * After `limit_ns` it gives up and writes CALIBATT_E_TIMEOUT to dev_status.
  * Lets a caller check the timeout path without faulting or hanging a GPU.
+ * Errors: CALIBATT_E_INVALID for a NULL dev_status or a limit outside
+ * (0, 10 s].
  */
 int calibatt_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status,
                                    calibatt_stream_t stream);
