@@ -193,6 +193,37 @@ def test_timestep_sharing_validation(lib):
     assert lib.calibatt_share_masks(fake, 2, 4, 3, 8, 8, fake, 9, fake, None) == _lib.E_INVALID
 
 
+def test_documented_errors_of_the_auxiliary_calls(lib):
+    # every case is refused on the host, before any launch
+    fake = ctypes.c_void_p(0x10000)
+    # one block per (run, head): n_runs * H above 65535 is unsupported
+    assert lib.calibatt_share_masks(fake, 1024, 64, 2, 8, 8, fake, 40000, fake, None) == _lib.E_UNSUPPORTED
+    # L * T above 2^20
+    run = (ctypes.c_int32 * 1)()
+    n = ctypes.c_int32(0)
+    assert lib.calibatt_timestep_clusters(fake, 2048, 1024, 1, 8, 8, 0.5, run, ctypes.byref(n), fake, 1 << 30,
+                                          None) == _lib.E_UNSUPPORTED
+    bl = _blocklist(4, 8, 8, 128, 128)
+    kept = ctypes.c_int64(0)
+    assert lib.calibatt_blocklist_kept(None, 0, 1, ctypes.byref(kept), fake, 8, None) == _lib.E_INVALID
+    assert lib.calibatt_blocklist_kept(ctypes.byref(bl), 3, 2, ctypes.byref(kept), fake, 8, None) == _lib.E_INVALID
+    assert lib.calibatt_blocklist_kept(ctypes.byref(bl), -1, 2, ctypes.byref(kept), fake, 8, None) == _lib.E_INVALID
+    assert lib.calibatt_blocklist_kept(ctypes.byref(bl), 0, 2, ctypes.byref(kept), fake, 4, None) == \
+        _lib.E_WORKSPACE
+    assert lib.calibatt_blocklist_kept(ctypes.byref(bl), 0, 2, ctypes.byref(kept), ctypes.c_void_p(0x10004), 8,
+                                       None) == _lib.E_INVALID
+    csr, pool = ctypes.c_int64(0), ctypes.c_int64(0)
+    assert lib.calibatt_blocklist_bytes(2, 8, 10, 0, 4, ctypes.byref(csr), ctypes.byref(pool)) == _lib.E_INVALID
+    assert lib.calibatt_blocklist_bytes(2, 8, -1, 3, 4, ctypes.byref(csr), ctypes.byref(pool)) == _lib.E_INVALID
+    # the sizes themselves: int64 row pointers + int16 columns; int32 base and pattern id per row, int32 pattern
+    # pointers, int16 offsets
+    assert lib.calibatt_blocklist_bytes(2, 8, 10, 3, 4, ctypes.byref(csr), ctypes.byref(pool)) == _lib.OK
+    assert (csr.value, pool.value) == (17 * 8 + 10 * 2, 16 * 8 + 4 * 4 + 4 * 2)
+    assert lib.calibatt_selftest_wait_timeout(10_000_000_001, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_merge_intervals(fake, 2, -1, 8, fake, fake, None) == _lib.E_INVALID
+    assert lib.calibatt_gather_rows(fake, fake, fake, 0, 4, 4, 256, None) == _lib.E_INVALID
+
+
 def test_skiplist_validation(lib):
     fake = ctypes.c_void_p(0x10000)
     assert lib.calibatt_interval_counts(None, 2, 8, 8, fake, None) == _lib.E_INVALID
