@@ -193,6 +193,29 @@ def test_energy_brute_force():
             assert E[0, qb, kb] == pytest.approx(tot / len(rows), abs=1e-13)
 
 
+def test_energy_non_square_blocks_brute_force_and_closed_form():
+    # Table S6 key grids: key blocks of a size other than the query block's,
+    # a ragged last key block, and a key grid of ceil(N / block_k) blocks
+    # that ignores the query padding (N = 10, Np = 12, 3-key blocks -> 4).
+    N, bq, bk, d, scale = 10, 4, 3, 3, 0.8
+    q = RNG.standard_normal((1, 12, d))
+    k = RNG.standard_normal((1, 12, d))
+    E = oracle.block_energy(q, k, N, bq, bk, scale)
+    assert E.shape == (1, 3, 4)
+    for qb in range(3):
+        rows = list(range(qb * bq, min(qb * bq + bq, N)))
+        for kb in range(4):
+            tot = 0.0
+            for i in rows:
+                s = [scale * math.fsum(q[0, i, t] * k[0, j, t] for t in range(d)) for j in range(N)]
+                z = math.fsum(math.exp(x) for x in s)
+                tot += math.fsum(math.exp(s[j]) / z for j in range(kb * bk, min(kb * bk + bk, N)))
+            assert E[0, qb, kb] == pytest.approx(tot / len(rows), abs=1e-13)
+    # q = 0: uniform attention, E[qb, kb] = (#real keys in kb) / N = 3, 3, 3, 1 tenths
+    E0 = oracle.block_energy(np.zeros_like(q), k, N, bq, bk, scale)
+    np.testing.assert_allclose(E0[0], np.broadcast_to([0.3, 0.3, 0.3, 0.1], (3, 4)), atol=1e-15)
+
+
 # ----------------------------------------------------------------- O3 select
 
 def test_topk_count_and_brute_force_order():
