@@ -24,9 +24,9 @@ import torch
 def gather_in_order(local, group=None):
     """All-gathers each rank's list of equally shaped tensors; returns the
     concatenation in rank order (rank 0's tensors first).  Ranks may hold
-    different counts, including none (then ``like`` must come from another
-    rank: every rank needs at least the shape, so pass a list with at least
-    one tensor on every rank)."""
+    different counts, but at least one tensor each: every rank takes the
+    shape of the padded exchange from its own first tensor (ValueError
+    otherwise)."""
     import torch.distributed as dist
     if not local:
         raise ValueError("every rank needs at least one tensor")
