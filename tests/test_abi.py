@@ -23,6 +23,24 @@ def declared_functions():
     return sorted(names)
 
 
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    # tests/c/abi_host.c: the header as C99 with strict warnings, linked
+    # against the library, host-only calls answered from C
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    pkg = Path(_lib.LIB_PATH).parent
+    exe = tmp_path / "abi_host"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", f"-I{HEADER.parent}",
+                    str(Path(__file__).resolve().parent / "c" / "abi_host.c"), f"-L{pkg}", "-lcalibatt",
+                    f"-Wl,-rpath,{pkg}", "-o", str(exe)], check=True, timeout=120)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
+
+
 def test_header_and_binding_agree():
     names = declared_functions()
     assert len(names) >= 14
